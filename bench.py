@@ -1,0 +1,518 @@
+"""Benchmark of the HiLS-Attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hils|reference] [--quick]
+
+Headline (`value`): prefill throughput in tokens/s on the prefill workload (B4 T8192 Hq16 Hkv4 d128
+S64 k16 W512, bf16). One step = one pass of the prefill hot path over the batch: landmark summaries
+(hils_chunk_summary), retrieval + GQA top-k (hils_select_topk) and Eq. 10 attention (hils_attn_fwd),
+inputs resident in HBM, L2 flushed (a 256 MiB write) between timed steps and outside the events.
+The same JSON line carries the decode workload (B8, 512K-token cache, 256 steps in a CUDA graph,
+us/token), the context-length sweep, the training step (forward + backward, B2 T8192), a roofline
+object per block, the end-to-end number through the public API with host buffers, the oracle's CPU
+time on a bounded sample, and the SM clocks sampled during the timed region.
+
+Multi-GPU (torchrun, one process per GPU): the batch is independent across sequences, so every rank
+runs its own batch (different seed) with no data-path collective: weak scaling; `value` = tokens of
+all ranks / max over ranks of the device time.
+--impl reference times the fp64 CPU oracle (the reference arm for this method) on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from chunk_wise_hierarchical_summary_b200 import workloads as W  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) of SM clock and throttle reasons during a timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu_index), "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+class Dist:
+    def __init__(self, n_gpus: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+            if backend == "nccl":
+                torch.cuda.set_device(self.local_rank)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            if torch.cuda.is_available():
+                self.pg.barrier(device_ids=[self.local_rank])
+            else:
+                self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if self.pg is None:
+            return x
+        dev = torch.device("cuda", self.local_rank) if torch.cuda.is_available() else torch.device("cpu")
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+def physical_gpu_index(local_rank: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids) and ids[local_rank].strip().isdigit():
+            return int(ids[local_rank])
+    return local_rank
+
+
+def timed_steps(steps, fn_stages, warmup, flush, dist: Dist, sampler=None):
+    """Run `warmup` untimed steps, then `steps` timed ones. fn_stages() launches one step and returns
+    nothing; stage boundaries are marked by the callback `mark` it receives. Returns per-stage device
+    milliseconds summed over the timed steps (list) and the total."""
+    for _ in range(warmup):
+        fn_stages(lambda: None)
+        if flush is not None:
+            flush.zero_()
+    torch.cuda.synchronize()
+    dist.barrier()
+    if sampler:
+        sampler.start()
+    records = []
+    for _ in range(steps):
+        if flush is not None:
+            flush.zero_()
+        evs = [torch.cuda.Event(enable_timing=True)]
+        evs[0].record()
+
+        def mark():
+            e = torch.cuda.Event(enable_timing=True)
+            e.record()
+            evs.append(e)
+
+        fn_stages(mark)
+        records.append(evs)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    n_stage = len(records[0]) - 1
+    stage_ms = [sum(r[i].elapsed_time(r[i + 1]) for r in records) for i in range(n_stage)]
+    return stage_ms, sum(stage_ms), clocks
+
+
+# ----------------------------------------------------------------------------- algorithmic work
+
+def window_left(p, Wn, S):
+    return (max(0, p - Wn + 1) // S) * S
+
+
+def prefill_work(w: W.Workload):
+    """Algorithmic flops of the prefill hot path and of each stage, from the sizes alone.
+    attention: 4 d flops per (query row, head, attended token) (QK^T and PV), attended = window + selected
+    chunk tokens; routing: 2 d per (row, head, candidate chunk); summaries: 4 S d per (head, chunk)."""
+    attended = 0
+    cand = 0
+    for p in range(w.q_pos0, w.q_pos0 + w.T):
+        l = window_left(p, w.W, w.S)
+        n = l // w.S
+        attended += (p - l + 1) + min(w.topk, n) * w.S
+        cand += n
+    rows = w.B * w.Hq
+    attn = 4 * w.d * attended * rows
+    route = 2 * w.d * cand * rows
+    summ = 4 * w.S * w.d * w.Nc * w.B * w.Hq
+    el = 2 if w.dtype == "bf16" else 4
+    attn_bytes = el * (w.B * w.Hq * w.T * w.d * 3 + w.B * w.Hkv * w.L * w.d * 2) + 4 * w.B * w.Hq * w.T \
+        + (el * w.d + 4) * w.B * w.Hq * w.Nc
+    return {"attn_flops": attn, "route_flops": route, "summary_flops": summ, "attn_bytes": attn_bytes,
+            "avg_attended": attended / w.T}
+
+
+def decode_bytes(w: W.Workload):
+    """Bytes one decode step must touch: every candidate summary (k' in the input dtype + fp32 b'),
+    the selected chunks' K and V, the window's K and V, q, q^ and the output."""
+    el = 2 if w.dtype == "bf16" else 4
+    p = w.L - 1
+    l = window_left(p, w.W, w.S)
+    n = l // w.S
+    summ = w.B * w.Hq * n * (w.d * el + 4)
+    chunks = w.B * w.Hkv * min(w.topk, n) * w.S * w.d * el * 2
+    win = w.B * w.Hkv * (p - l + 1) * w.d * el * 2
+    io = w.B * w.Hq * w.d * el * 3 + w.B * w.Hq * 4
+    return {"total": summ + chunks + win + io, "summaries": summ, "chunks": chunks, "window": win, "io": io}
+
+
+# ----------------------------------------------------------------------------- GPU arms
+
+def bench_prefill(args, dist, dev, H, peaks):
+    w = W.PREFILL_BF16
+    x = W.prefill_inputs(w, seed=1000 + dist.rank, device=dev)
+    k_sum = torch.empty((w.B, w.Hq, w.Nc, w.d), dtype=torch.bfloat16, device=dev)
+    b_sum = torch.empty((w.B, w.Hq, w.Nc), dtype=torch.float32, device=dev)
+    idx = torch.empty((w.B, w.Hkv, w.T, w.topk), dtype=torch.int32, device=dev)
+    out = torch.empty_like(x["q"])
+    lse = torch.empty((w.B, w.Hq, w.T), dtype=torch.float32, device=dev)
+    p = H.make_params(w.B, w.T, w.L, w.Hq, w.Hkv, w.d, w.S, w.topk, w.W)
+    nws = H.workspace_size(p, H.OP_ATTN_FWD)
+    ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(mark):
+        H.chunk_summary(x["k"], x["q_land"], w.S, k_sum=k_sum, b_sum=b_sum)
+        mark()
+        H.select_topk(x["q_hat"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S, topk=w.topk, window=w.W, idx=idx)
+        mark()
+        H.attn_fwd(x["q"], x["k"], x["v"], x["q_hat"], k_sum, b_sum, idx, S=w.S, window=w.W, out=out, lse=lse,
+                   workspace=ws if nws else None)
+        mark()
+
+    sampler = ClockSampler(physical_gpu_index(dist.local_rank))
+    stage_ms, total_ms, clocks = timed_steps(args.steps, step, args.warmup, flush, dist, sampler)
+    work = prefill_work(w)
+    attn_s = stage_ms[2] / args.steps / 1e3
+    achieved = work["attn_flops"] / attn_s / 1e12
+    # union ratio of the selections (chunks a 32-query tile must visit / chunks each query selects)
+    res = {
+        "workload": w, "x": x, "out": out, "lse": lse, "idx": idx, "stage_ms": [s / args.steps for s in stage_ms],
+        "ms_per_step": total_ms / args.steps, "clocks": clocks, "work": work,
+        "roofline": {"bound": "tensor", "kernel": "hils_attn_fwd", "achieved": achieved,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": None,
+                     "note": "algorithmic flops = 4*d per (row, head, attended token); attended = window + "
+                             "selected chunk tokens, %.1f per query on average" % work["avg_attended"]},
+        "launches_per_step": 3,
+    }
+    del flush
+    return res
+
+
+def bench_prefill_e2e(args, dist, dev, H, res):
+    """Same metric through the public API with host buffers: every step copies the inputs from pinned
+    host memory, runs the three calls and copies out + lse back."""
+    w = res["workload"]
+    xh = {n: res["x"][n].cpu().pin_memory() for n in ("q", "k", "v", "q_hat", "q_land")}
+    xd = {n: torch.empty_like(res["x"][n]) for n in xh}
+    out_h = torch.empty(res["out"].shape, dtype=res["out"].dtype).pin_memory()
+    lse_h = torch.empty(res["lse"].shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in xh.values())
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * 4
+    steps = max(1, min(args.steps, 10))
+
+    def step(mark):
+        for n in xh:
+            xd[n].copy_(xh[n], non_blocking=True)
+        out, lse, _, _, _ = H.prefill(xd["q"], xd["k"], xd["v"], xd["q_hat"], xd["q_land"], S=w.S, topk=w.topk,
+                                      window=w.W)
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+        mark()
+
+    _, total_ms, _ = timed_steps(steps, step, 2, None, dist)
+    ms = dist.max(total_ms / steps)
+    return {"value": dist.world * w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def bench_decode(args, dist, dev, H, peaks, w: W.Workload, steps: int):
+    x = W.decode_inputs(w, seed=2000 + dist.rank, device=dev)
+    k_sum, b_sum = H.chunk_summary(x["k_cache"], x["q_land"], w.S)
+    out = torch.empty_like(x["q"])
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    idx = torch.empty((w.B, w.Hkv, w.topk), dtype=torch.int32, device=dev)
+    p = H.make_params(w.B, 1, w.L, w.Hq, w.Hkv, w.d, w.S, w.topk, w.W, w.L - 1)
+    ws = torch.empty(H.workspace_size(p, H.OP_DECODE), dtype=torch.uint8, device=dev)
+
+    def one():
+        H.decode(x["q"], x["q_hat"], x["k_cache"], x["v_cache"], k_sum, b_sum, S=w.S, topk=w.topk, window=w.W,
+                 out=out, lse=lse, idx_out=idx, workspace=ws)
+
+    # capture `steps` decode steps in one CUDA graph (the per-step footprint exceeds L2: no flush)
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            one()
+    torch.cuda.current_stream(dev).wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(steps):
+            one()
+
+    def run(mark):
+        graph.replay()
+        mark()
+
+    _, total_ms, clocks = timed_steps(1, run, max(1, args.warmup // 3), None, dist,
+                                      ClockSampler(physical_gpu_index(dist.local_rank)))
+    needles_found = 0
+    for b in range(w.B):
+        needles_found += len(set(x["needle_chunks"][b].tolist()) & set(idx[b, 0].tolist()))
+    ms_step = total_ms / steps
+    nbytes = decode_bytes(w)
+    gbs = nbytes["total"] / (ms_step / 1e3) / 1e9
+    del graph
+    return {"workload": w.name, "us_per_token": ms_step * 1e3, "us_per_step_per_seq": ms_step * 1e3 / w.B,
+            "steps": steps, "bytes_per_step": nbytes,
+            "roofline": {"bound": "hbm", "kernel": "hils_decode (whole step: score, select, attend, combine)",
+                         "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                         "traffic": None},
+            "needle_recall": needles_found / max(1, w.B * min(w.needles, w.Nc)), "clocks": clocks,
+            "launches_per_step": 4}
+
+
+def bench_train(args, dist, dev, H, peaks):
+    w = W.TRAIN_BF16
+    x = W.prefill_inputs(w, seed=3000 + dist.rank, device=dev, with_dout=True)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(mark):
+        out, lse, idx, k_sum, b_sum = H.prefill(x["q"], x["k"], x["v"], x["q_hat"], x["q_land"], S=w.S,
+                                                topk=w.topk, window=w.W)
+        mark()
+        H.attn_bwd(x["q"], x["k"], x["v"], x["q_hat"], x["q_land"], k_sum, b_sum, idx, out, lse, x["dout"], S=w.S,
+                   window=w.W)
+        mark()
+
+    steps = max(1, min(args.steps, 5))
+    stage_ms, total_ms, _ = timed_steps(steps, step, 1, flush, dist)
+    work = prefill_work(w)
+    fwd_flops = work["attn_flops"] + work["route_flops"] + work["summary_flops"]
+    bwd_flops = work["attn_flops"] * 14 // 4 + 2 * work["summary_flops"]
+    ms = total_ms / steps
+    return {"workload": w.name, "tokens_per_s": w.B * w.T / (ms / 1e3), "ms_per_step": ms,
+            "fwd_ms": stage_ms[0] / steps, "bwd_ms": stage_ms[1] / steps,
+            "roofline": {"bound": "tensor", "kernel": "hils_attn_bwd",
+                         "achieved": bwd_flops / (stage_ms[1] / steps / 1e3) / 1e12,
+                         "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                         "frac": bwd_flops / (stage_ms[1] / steps / 1e3) / 1e12 / peaks["bf16_tflops_sustained"],
+                         "traffic": None, "note": "bwd flops = 14*d per (row, head, attended token) + summary bwd"},
+            "launches_per_step": 5}
+
+
+# ----------------------------------------------------------------------------- CPU (oracle)
+
+def oracle_prefill_sample(x_cpu, w: W.Workload, groups, row_blocks, block_rows, budget_s=None):
+    """The oracle on a bounded sample of the prefill workload: for each listed (b, KV group), all of
+    its summaries, then selection + attention for up to `row_blocks` evenly spaced blocks of
+    `block_rows` query rows (visited in a stratified order, stopping once `budget_s` seconds have
+    passed). Returns (seconds, equivalent tokens = rows * G / Hq, blocks done)."""
+    import oracle
+    from oracle import Geometry
+
+    def np64(t):
+        return t.to(torch.float64).numpy()
+
+    order = sorted(range(row_blocks), key=lambda r: int(format(r, "016b")[::-1], 2))  # bit-reversal strata
+    rows_done, blocks_done = 0, 0
+    t0 = time.perf_counter()
+    for b, grp in groups:
+        hs = slice(grp * w.G, (grp + 1) * w.G)
+        kk = np64(x_cpu["k"][b:b + 1, grp:grp + 1])
+        vv = np64(x_cpu["v"][b:b + 1, grp:grp + 1])
+        g1 = Geometry(B=1, T=1, L=w.L, Hq=w.G, Hkv=1, d=w.d, S=w.S, topk=w.topk, W=w.W)
+        ks, bs = oracle.chunk_summary(g1, kk, np64(x_cpu["q_land"][b:b + 1, hs]))
+        for r in order:
+            if budget_s is not None and blocks_done > 0 and time.perf_counter() - t0 > budget_s:
+                break
+            r0 = int((w.T - block_rows) * (r + 0.5) / row_blocks)
+            gr = Geometry(B=1, T=block_rows, L=w.L, Hq=w.G, Hkv=1, d=w.d, S=w.S, topk=w.topk, W=w.W, q_pos0=r0)
+            rows = slice(r0, r0 + block_rows)
+            qh = np64(x_cpu["q_hat"][b:b + 1, hs, rows])
+            idx, _ = oracle.select_topk(gr, qh, ks, bs)
+            oracle.attn_fwd(gr, np64(x_cpu["q"][b:b + 1, hs, rows]), kk, vv, qh, ks, bs, idx)
+            rows_done += block_rows
+            blocks_done += 1
+    secs = time.perf_counter() - t0
+    return secs, rows_done * w.G / w.Hq, blocks_done
+
+
+def cpu_baseline(x_gpu, w, budget_s=10.0):
+    import oracle
+
+    x_cpu = {n: x_gpu[n][:1].cpu() for n in ("q", "k", "v", "q_hat", "q_land")}
+    secs, tokens, blocks = oracle_prefill_sample(x_cpu, w, [(0, 0)], 64, 128, budget_s=budget_s)
+    return {"value": tokens / secs, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"batch 0, KV group 0 ({w.G} query heads, all {w.Nc} chunk summaries) and {blocks} of 64 "
+                      f"stratified blocks of 128 query rows, stopped after ~{budget_s:.0f} s; tokens counted as "
+                      f"rows*G/Hq; {secs:.1f} s of CPU time"}
+
+
+def run_reference(args, dist):
+    """Reference arm: the fp64 CPU oracle on a bounded sample of the prefill workload, per step."""
+    if dist.rank != 0:
+        return
+    import oracle
+
+    w = W.PREFILL_BF16
+    x = W.prefill_inputs(w, seed=1000, device="cpu")
+    groups, blocks, rows = [(0, 0)], 2, 32
+    for _ in range(args.warmup):
+        oracle_prefill_sample(x, w, groups, blocks, rows)
+    total, tokens = 0.0, 0.0
+    for _ in range(args.steps):
+        s, t, _ = oracle_prefill_sample(x, w, groups, blocks, rows)
+        total += s
+        tokens += t
+    value = tokens / total
+    sample = (f"1 (batch, KV group) slice x {blocks} blocks of {rows} query rows per step; tokens = rows*G/Hq")
+    line = {"metric": "HiLS prefill tokens/s (B4 T8192 Hq16 Hkv4 d128 S64 k16 W512)", "value": value,
+            "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.T, "parallelism": "cpu oracle"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="hils", choices=("hils", "reference"))
+    ap.add_argument("--quick", action="store_true", help="headline only (no decode sweep / training blocks)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    dist = Dist(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, dist)
+            return
+        import chunk_wise_hierarchical_summary_b200.hils as H
+
+        dev = torch.device("cuda", dist.local_rank)
+        torch.cuda.set_device(dev)
+        peaks, peak_src = load_peaks()
+        pre = bench_prefill(args, dist, dev, H, peaks)
+        w = pre["workload"]
+        ms = dist.max(pre["ms_per_step"])
+        value = dist.world * w.B * w.T / (ms / 1e3)
+        e2e = bench_prefill_e2e(args, dist, dev, H, pre)
+        decode = bench_decode(args, dist, dev, H, peaks, W.DECODE_BF16, 256)
+        extra = {}
+        if not args.quick:
+            extra["decode_sweep"] = []
+            for L in W.DECODE_SWEEP_L:
+                r = bench_decode(args, dist, dev, H, peaks, W.decode_sweep(L), 64)
+                extra["decode_sweep"].append({"L": L, "us_per_token": r["us_per_token"],
+                                              "bytes_per_step": r["bytes_per_step"]["total"],
+                                              "hbm_frac": r["roofline"]["frac"], "needle_recall": r["needle_recall"]})
+            extra["train"] = bench_train(args, dist, dev, H, peaks)
+        cpu = None
+        if dist.world == 1:
+            cpu = cpu_baseline(pre["x"], w)
+        launches = pre["launches_per_step"] * args.steps
+        line = {
+            "metric": "HiLS prefill tokens/s (B4 T8192 Hq16 Hkv4 d128 S64 k16 W512); decode us/token at 512K ctx in "
+                      "'decode'; % of TC/HBM roofline",
+            "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "global_batch": w.B * dist.world, "seq_len": w.T,
+                       "parallelism": f"dp{dist.world} (independent sequences per GPU)",
+                       "l2": "flushed (256 MiB write) between timed steps, outside the events",
+                       "peaks": peak_src},
+            "stage_ms": {"chunk_summary": pre["stage_ms"][0], "select_topk": pre["stage_ms"][1],
+                         "attn_fwd": pre["stage_ms"][2]},
+            "roofline": pre["roofline"],
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": pre["clocks"],
+            "decode": decode,
+            **extra,
+        }
+        if dist.rank == 0:
+            print(json.dumps(line, default=lambda o: getattr(o, "name", str(o))))
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,105 @@
+// Device-side helpers shared by the HiLS kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hils.h"
+
+namespace hils {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Sizes of one problem, resolved on the host (tau filled in, derived counts computed).
+struct Dims {
+    int B, T, L, Hq, Hkv, d, S, topk, W, q_pos0;
+    int G, Nc;
+    float tau;
+};
+
+__host__ __device__ __forceinline__ int window_left(int pos, int W, int S) {
+    int e = pos - W + 1;
+    if (e < 0) e = 0;
+    return (e / S) * S;
+}
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+
+// Float -> uint32 whose unsigned order equals the float order (for radix / sort keys).
+__device__ __forceinline__ uint32_t float_order_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float float_from_order_key(uint32_t k) {
+    uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+    return __uint_as_float(u);
+}
+
+// Sort key that orders by (value descending, index ascending) under an ascending 64-bit sort.
+__device__ __forceinline__ uint64_t desc_value_key(float v, uint32_t index) {
+    return ((uint64_t)(~float_order_key(v)) << 32) | (uint64_t)index;
+}
+__device__ __forceinline__ float desc_key_value(uint64_t key) { return float_from_order_key(~(uint32_t)(key >> 32)); }
+__device__ __forceinline__ uint32_t desc_key_index(uint64_t key) { return (uint32_t)key; }
+
+// Ascending bitonic sort of n (a power of two) 64-bit keys in shared memory by the whole block.
+__device__ __forceinline__ void block_bitonic_sort(uint64_t *keys, int n) {
+    for (int size = 2; size <= n; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            __syncthreads();
+            for (int t = threadIdx.x; t < (n >> 1); t += blockDim.x) {
+                int lo = 2 * t - (t & (stride - 1));
+                int hi = lo + stride;
+                bool up = ((lo & size) == 0);
+                uint64_t a = keys[lo], b = keys[hi];
+                if ((a > b) == up) { keys[lo] = b; keys[hi] = a; }
+            }
+        }
+    }
+    __syncthreads();
+}
+
+__host__ __device__ __forceinline__ int next_pow2(int n) {
+    int p = 1;
+    while (p < n) p <<= 1;
+    return p;
+}
+
+// Load `n` consecutive elements (n a multiple of 8 for bf16, 4 for fp32; 16-byte aligned) as floats.
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float *out) {
+    uint4 raw = *reinterpret_cast<const uint4 *>(p);
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        float2 f = __bfloat1622float2(h[t]);
+        out[2 * t] = f.x;
+        out[2 * t + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void load8(const float *p, float *out) {
+    float4 a = *reinterpret_cast<const float4 *>(p);
+    float4 b = *reinterpret_cast<const float4 *>(p + 4);
+    out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+    out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
+}
+
+}  // namespace hils

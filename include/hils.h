@@ -1,0 +1,166 @@
+/*
+ * hils.h — C ABI of the HiLS-Attention hot path on NVIDIA B200 (sm_100a).
+ *
+ * Method: "Hierarchical Sparse Attention Done Right: Toward Infinite Context Modeling"
+ * (arXiv 2607.02980). Four stages: (a) landmark chunk summaries (Eq. 8), (b) retrieval scores
+ * (Eq. 7) and GQA-shared top-k chunk selection (Sec. 3 RQ1, Sec. 4 "GQA"), (c) softmax attention of
+ * each query within each selected chunk and within its chunk-aligned causal sliding window
+ * (Sec. 2), (d) fusion of the per-chunk outputs by softmax(s^) over the selected chunks plus the
+ * window (Eq. 10), in prefill, single-token decode and backward forms.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Sizes (hils_params): B batch, T query rows, L KV length, Hq query heads, Hkv KV heads
+ * (G = Hq/Hkv heads share one KV head: query head h reads KV head h/G), d head dim, S chunk size,
+ * topk chunks kept per query, window W, q_pos0 = absolute position of query row 0 (row i sits at
+ * p = q_pos0 + i and attends keys at positions <= p), scale tau (0 => 1/sqrt(d)).
+ * Nc = floor(L/S) complete chunks; chunk c holds tokens [c*S, (c+1)*S).
+ * Window of position p: tokens [l_p, p] with l_p = S*floor(max(0, p-W+1)/S); its candidate chunks
+ * are c < n_p = l_p/S (the chunks wholly left of the window; all complete).
+ *
+ * Tensors are dense, row-major, contiguous, 16-byte aligned device pointers:
+ *   q, q_hat, out, dout, dq, dq_hat        [B, Hq, T, d]   element type = params.dtype
+ *   k, v, dk, dv (prefill) / k_cache, v_cache [B, Hkv, L, d]   params.dtype
+ *   q_land, dq_land                         [B, Hq, Nc, d]  params.dtype (one landmark query per chunk)
+ *   k_sum                                   [B, Hq, Nc, d]  params.dtype (summary key k')
+ *   b_sum                                   [B, Hq, Nc]     float32      (entropy bias b')
+ *   idx                                     [B, Hkv, T, topk] int32 (ascending chunk ids, -1 padded)
+ *   lse                                     [B, Hq, T]      float32 (natural-log log Z^_i)
+ * An idx row is read as a set: entries outside [0, n_p) are ignored and a repeated id counts once.
+ *
+ * Ownership: the caller owns every buffer, including the workspace (size from
+ * hils_workspace_size). The library keeps no state between calls. Every compute call is
+ * asynchronous on `stream` and returns after enqueueing its kernels.
+ * Errors: shapes, pointers, alignment and workspace size are checked before any launch
+ * (HILS_ERR_INVALID_ARG / HILS_ERR_UNSUPPORTED / HILS_ERR_WORKSPACE, nothing enqueued); a failed
+ * launch returns HILS_ERR_CUDA. hils_last_error() gives a thread-local message. No C++ exception
+ * crosses this boundary.
+ */
+#ifndef HILS_H_
+#define HILS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HILS_API __attribute__((visibility("default")))
+#else
+#define HILS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *hils_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+    HILS_OK = 0,
+    HILS_ERR_INVALID_ARG = 1, /* bad size, null or misaligned pointer */
+    HILS_ERR_UNSUPPORTED = 2, /* valid but outside what the kernels implement (e.g. d not 64/128) */
+    HILS_ERR_WORKSPACE = 3,   /* workspace missing or smaller than hils_workspace_size() */
+    HILS_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+    HILS_ERR_TIMEOUT = 5      /* a bounded device-side wait expired (reported by hils_check) */
+} hils_status;
+
+typedef enum { HILS_BF16 = 0, HILS_FP32 = 1 } hils_dtype;
+
+typedef struct {
+    int32_t B, T, L, Hq, Hkv, d, S, topk, window;
+    int32_t q_pos0;   /* absolute position of query row 0: 0 for prefill, L-1 for decode */
+    float scale;      /* tau; 0 => 1/sqrt(d) */
+    int32_t dtype;    /* hils_dtype of q, k, v, q_hat, q_land, k_sum, out and the gradients */
+} hils_params;
+
+/* Operation ids for hils_workspace_size. */
+enum { HILS_OP_SUMMARY = 0, HILS_OP_SELECT = 1, HILS_OP_ATTN_FWD = 2, HILS_OP_DECODE = 3, HILS_OP_ATTN_BWD = 4 };
+
+/* Supported ranges (HILS_ERR_UNSUPPORTED outside them). */
+#define HILS_MAX_S 128
+#define HILS_MAX_TOPK 64
+
+/*
+ * Bytes of device workspace `op` needs for these sizes (0 = none; the pointer may then be NULL).
+ * Returns (size_t)-1 if the sizes are invalid. Host-only, no CUDA call.
+ */
+HILS_API size_t hils_workspace_size(const hils_params *p, int op);
+
+/*
+ * Stage (a), Eq. 8 (Prop. 3.1, the landmark summary): for every b, query head h and complete chunk
+ * c in [c_begin, c_end):  u_j = tau * q_land[b,h,c] . k[b,h/G,c*S+j],  p = softmax_j(u),
+ *   k_sum[b,h,c] = sum_j p_j k_j  (stored in params.dtype),  b_sum[b,h,c] = -sum_j p_j log p_j.
+ * Chunks outside the range are not touched, so a decode cache can be extended as chunks complete.
+ * Uses q_land/k_sum/b_sum sized by Nc = floor(L/S); 0 <= c_begin <= c_end <= Nc. T, topk, window
+ * and q_pos0 are not read. An empty range returns HILS_OK without reading any pointer. No workspace.
+ */
+HILS_API hils_status hils_chunk_summary(const hils_params *p, const void *k, const void *q_land, int32_t c_begin,
+                               int32_t c_end, void *k_sum, float *b_sum, hils_stream_t stream);
+
+/*
+ * Stage (b), Eq. 7 + Sec. 3 RQ1 + Sec. 4 "GQA": for every (b, KV group g, row i) with n = n_p
+ * candidates:  s^_{h,c} = tau * q_hat[b,h,i] . k_sum[b,h,c] + b_sum[b,h,c]  for c < n and each head h
+ * of the group; group score g_c = max_h (s^_{h,c} - LSE_{c'<n} s^_{h,c'}); keep the min(topk, n)
+ * largest by (g_c desc, c asc). idx[b,g,i,:] = those ids ascending, then -1.
+ * gap (nullable, float32 [B, Hkv, T]) = g_(topk) - g_(topk+1), +inf when n <= topk.
+ * Scores in fp32. Supports G * Nc * 4 + next_pow2(Nc) * 8 <= 200 KiB of shared memory per row
+ * (Nc <= 8192 at G = 4); longer contexts use hils_decode. Workspace: none.
+ */
+HILS_API hils_status hils_select_topk(const hils_params *p, const void *q_hat, const void *k_sum, const float *b_sum,
+                             int32_t *idx, float *gap, void *workspace, size_t workspace_bytes,
+                             hils_stream_t stream);
+
+/*
+ * Stages (c)+(d), Eq. 10 (chunked prefill form): for every (b, h, row i) at position p:
+ *   window logits s_j = tau q.k_j, j in [l_p, p];  for each selected chunk c (idx, as a set):
+ *   s^_c (as above), L_c = LSE_{j in c} s_j, o_c = sum_j exp(s_j - L_c) v_j;
+ *   lse = log Z^ = LSE({s_j}_window U {s^_c}_selected);
+ *   out = sum_window exp(s_j - lse) v_j + sum_c exp(s^_c - lse) o_c.
+ * The per-chunk outputs o_c never reach memory: each chunk's weights are scaled by
+ * exp(s^_c - L_c) before its value product. fp32 accumulation. Workspace: none.
+ */
+HILS_API hils_status hils_attn_fwd(const hils_params *p, const void *q, const void *k, const void *v, const void *q_hat,
+                          const void *k_sum, const float *b_sum, const int32_t *idx, void *out, float *lse,
+                          void *workspace, size_t workspace_bytes, hils_stream_t stream);
+
+/*
+ * One decode step (stages b-d for T = 1 at position q_pos0 = L-1 over a KV cache of L tokens):
+ * scores every candidate chunk's summary, selects topk chunks per KV group as hils_select_topk
+ * does, attends, and fuses as hils_attn_fwd does. q, q_hat [B, Hq, 1, d]; out [B, Hq, 1, d];
+ * lse [B, Hq]; idx_out (nullable) [B, Hkv, topk]. Requires T == 1 and q_pos0 == L-1.
+ * Workspace: hils_workspace_size(p, HILS_OP_DECODE) bytes.
+ */
+HILS_API hils_status hils_decode(const hils_params *p, const void *q, const void *q_hat, const void *k_cache,
+                        const void *v_cache, const void *k_sum, const float *b_sum, void *out, float *lse,
+                        int32_t *idx_out, void *workspace, size_t workspace_bytes, hils_stream_t stream);
+
+/*
+ * Backward of hils_chunk_summary + hils_attn_fwd for loss = sum(dout * out), idx held fixed (the
+ * hard top-k is not differentiable; gradients reach q_land through s^ -> k_sum, b_sum -> Eq. 8):
+ *   window: ds_j = a_j (dout.v_j - D), dv_j += a_j dout,  a_j = exp(s_j - lse), D = dout.out
+ *   chunk:  ds^_c = b_c (dout.o_c - D), ds_j = b_c pi_cj (dout.v_j - dout.o_c), dv_j += b_c pi_cj dout
+ *   dq = tau sum ds_j k_j, dk_j += tau ds_j q, dq_hat = tau sum ds^_c k_sum_c,
+ *   dk_sum_c += tau ds^_c q_hat, db_sum_c += ds^_c;  Eq. 8 backward:
+ *   du_j = p_j (dk_sum.(k_j - k_sum) - db_sum (log p_j + b_sum)), dq_land = tau sum du_j k_j,
+ *   dk_j += p_j dk_sum + tau du_j q_land.
+ * out and lse must be this forward's outputs. Every gradient is fully overwritten (fp32
+ * accumulation, stored in params.dtype). Requires q_pos0 == 0 and T == L (self-attention prefill).
+ * Workspace: hils_workspace_size(p, HILS_OP_ATTN_BWD) bytes.
+ */
+HILS_API hils_status hils_attn_bwd(const hils_params *p, const void *q, const void *k, const void *v, const void *q_hat,
+                          const void *q_land, const void *k_sum, const float *b_sum, const int32_t *idx,
+                          const void *out, const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                          void *dq_hat, void *dq_land, void *workspace, size_t workspace_bytes,
+                          hils_stream_t stream);
+
+/* Waits for `stream`, then reports a device-side error word (HILS_ERR_TIMEOUT) or a CUDA error. */
+HILS_API hils_status hils_check(hils_stream_t stream);
+
+HILS_API const char *hils_status_string(hils_status s);
+HILS_API const char *hils_last_error(void); /* thread-local message for the last failing call */
+HILS_API const char *hils_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HILS_H_ */

