@@ -85,6 +85,10 @@ hils_status check_ws(const char *fn, void *ws, size_t have, size_t need) {
 }
 
 }  // namespace
+
+// Lets other translation units of the library set the thread-local message of hils_last_error().
+void record_error(const char *msg) { g_last_error = msg; }
+
 }  // namespace hils
 
 using namespace hils;

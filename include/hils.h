@@ -152,6 +152,30 @@ HILS_API hils_status hils_attn_bwd(const hils_params *p, const void *q, const vo
                           void *dq_hat, void *dq_land, void *workspace, size_t workspace_bytes,
                           hils_stream_t stream);
 
+/*
+ * A decode step that allocates nothing. The paper has no counterpart: this exists for callers that
+ * cannot hand the library a workspace (a serving engine whose memory planner owns the whole device
+ * and forbids library-side allocation, a foreign-language binding that passes tensor pointers but
+ * has no device allocator, a latency-critical loop that cannot afford cudaMalloc's implicit
+ * synchronisation). Same inputs, outputs, rules and results as hils_decode; the scratch lives in a
+ * static __device__ array of HILS_DECODE_NOALLOC_MAX_BYTES that every GPU loading this library
+ * holds until the process exits.
+ *  - Sizes whose decode workspace (hils_workspace_size(p, HILS_OP_DECODE)) exceeds the array are
+ *    rejected with HILS_ERR_UNSUPPORTED before anything is enqueued.
+ *  - The first call on a device (with that device current) looks up the array's device address
+ *    with cudaGetSymbolAddress; make that first call before any stream capture. Later calls reuse it.
+ *  - All calls on a device share the one array and it keeps the previous call's contents: calls
+ *    whose GPU work overlaps (e.g. on two streams without ordering between them) race and corrupt
+ *    each other's results; order them on one stream or with events. Every scratch byte a call reads
+ *    is written earlier in the same call, so nothing needs clearing between calls.
+ *  - No cudaMalloc, cudaFree or allocating library routine is called.
+ */
+#define HILS_DECODE_NOALLOC_MAX_BYTES (32u << 20)
+HILS_API hils_status hils_decode_noalloc(const hils_params *p, const void *q, const void *q_hat,
+                                         const void *k_cache, const void *v_cache, const void *k_sum,
+                                         const float *b_sum, void *out, float *lse, int32_t *idx_out,
+                                         hils_stream_t stream);
+
 /* Waits for `stream`, then reports a device-side error word (HILS_ERR_TIMEOUT) or a CUDA error. */
 HILS_API hils_status hils_check(hils_stream_t stream);
 
