@@ -8,5 +8,5 @@ cudaError_t launch_attn_fwd_tc(const Dims &, const void *, const void *, const v
                                const float *, const int *, void *, float *, cudaStream_t) {
     return cudaErrorNotSupported;
 }
-hils_status check_device_errors() { return HILS_OK; }
+
 }  // namespace hils

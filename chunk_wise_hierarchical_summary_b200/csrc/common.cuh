@@ -78,6 +78,19 @@ __device__ __forceinline__ void block_bitonic_sort(uint64_t *keys, int n) {
     __syncthreads();
 }
 
+// Number of SMs of the current device (cached per device ordinal).
+inline int num_sms() {
+    static int cache[256] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
 __host__ __device__ __forceinline__ int next_pow2(int n) {
     int p = 1;
     while (p < n) p <<= 1;

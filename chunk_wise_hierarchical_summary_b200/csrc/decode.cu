@@ -1,213 +1,444 @@
 // Single-token decode over a long KV cache: stages (b)-(d) for one query at position L-1
-// ("Hierarchical Sparse Attention Done Right", Eq. 7, Sec. 4 "GQA", Eq. 10).
+// ("Hierarchical Sparse Attention Done Right", Eq. 7, Sec. 3 RQ1, Sec. 4 "GQA", Eq. 10).
 //
-// Four launches, all HBM-streaming CUDA-core kernels (one query row per head: no dense contraction):
-//  1. score   grid (slices, Hkv, B): streams the summaries k'/b' of a slice of candidate chunks once,
-//             s^_{h,c} = tau q^_h . k'_{h,c} + b'_{h,c}; writes per (slice, head) the partial
-//             (max, sum exp) and the slice's top-(k+1) chunks by s^ (value desc, id asc).
-//  2. select  grid (Hkv, B): per-head LSE from the partials; group score g_c = max_h (s^_{h,c} - LSE_h)
-//             over the union of the lists; top-k by (g desc, c asc).
-//             Exactness: if c is in the group's top-(k+1), the head h* attaining g_c ranks c in its own
-//             top-(k+1) by s^ (any chunk above c there has a larger g), hence in its slice's list; and
-//             g_c is recovered from h*'s entry. So the union of per-slice per-head top-(k+1) lists holds
-//             the group's top-(k+1) with exact scores, and ranking the union by the per-entry maximum
-//             reproduces the full selection.
-//  3. attend  grid (tiles, Hkv, B): one S-token tile (a selected chunk or a window tile) per CTA, all G
-//             heads; writes a partial (max, sum, acc[d]) of the Eq. 10 online softmax over adjusted
-//             logits (chunk tokens carry s_j - L_c + s^_c).
-//  4. combine grid over (b, h): merges the tiles' partials into out and lse.
+// Three launches; one query row per head means no dense contraction, so these are HBM-streaming
+// CUDA-core kernels:
+//  1. score    grid (slices, Hq, B): each CTA pulls one 128-candidate slice of a head's summaries
+//              (32 KiB at d 128 bf16) into shared memory with a single TMA bulk copy, then computes
+//              s^_{h,c} = tau q^_h . k'_{h,c} + b'_{h,c} into a score buffer, plus the slice's partial
+//              (max, sum exp).
+//  2. select   grid (Hkv, B). Per-head LSE from the partials; group score g_c = max_h (s^_{h,c} - LSE_h)
+//              as order-preserving 32-bit keys; an MSB-first radix select (four byte passes, warp-
+//              aggregated shared-memory histogram) finds the k-th largest key; an ordered compaction
+//              keeps every larger key and the lowest-id equal keys (the tie rule); one warp sorts
+//              those k entries and writes the ids ascending.
+//  3. attend   grid (tiles, Hkv, B): one S-token tile (a selected chunk or a window tile) per CTA; K
+//              and V staged by TMA bulk copies; all G heads; a partial (max, sum, acc[d]) of the online
+//              softmax over adjusted logits (a chunk token carries s_j - L_c + s^_c, s^_c read from the
+//              score buffer). The last CTA of each (b, KV group) to finish (an atomic counter, no
+//              waiting) merges the group's partials into out and lse.
 #include "internal.h"
+#include "tma.cuh"
 
 namespace hils {
 namespace {
 
-constexpr int kScoreThreads = 256;
-constexpr int kSelThreads = 512;
-constexpr int kAttnThreads = 128;
-constexpr int kMaxSliceChunks = 8192;
-constexpr int kMaxListEntries = 8192;
+constexpr int kSelThreads = 256;
+constexpr int kSelPart = 1024;    // candidates per select CTA
+constexpr int kSelHeadsInFlight = 8;  // heads whose scores each select thread loads up front
+constexpr int kSelMerge = 4096;   // shared keys: a part, then the merged lists (nparts * topk <= this)
+constexpr int kAttnThreads = 256;
+
+// Device-side error word of this file (bit 0: a bounded wait expired). Read by decode_error_flags().
+__device__ unsigned int g_decode_errors = 0;
 
 struct DecodePlan {
-    int n;        // candidate chunks
-    int nslices;  // score slices per (b, g)
-    int per;      // chunks per slice
-    int K1;       // list length per (slice, head) = topk + 1
+    int n;        // candidate chunks of the query at L-1
+    int nslices;  // score slices per (b, head)
+    int per;      // candidates per slice
     int wtiles;   // window tiles
     int ntiles;   // topk + wtiles
-    size_t off_part, off_list, off_sel, off_attn, total;
+    int nparts;   // select CTAs per (b, KV group)
+    size_t off_scores, off_part, off_list, off_sel, off_attn, off_count, off_selcount, total;
 };
+
+constexpr int kSliceElems = 16384;  // summary elements per scored slice
+constexpr int kScorePartsPerSliceHost = 4;  // partials per slice (one per consumer warp of a slot)
 
 DecodePlan make_plan(const Dims &D) {
     DecodePlan P{};
     const int pos = D.L - 1;
     const int l = window_left(pos, D.W, D.S);
     P.n = l / D.S;
-    P.K1 = D.topk + 1;
-    int max_slices = kMaxListEntries / (D.G * P.K1);
-    if (max_slices < 1) max_slices = 1;
-    int want = (P.n + 255) / 256;
-    P.nslices = want < 1 ? 1 : (want > max_slices ? max_slices : want);
-    P.per = P.n > 0 ? (P.n + P.nslices - 1) / P.nslices : 0;
+    const int bg = D.B * D.Hkv;
+    P.per = kSliceElems / D.d;  // 128 rows at d 128
+    P.nslices = P.n > 0 ? (P.n + P.per - 1) / P.per : 1;
     P.wtiles = (pos - l + 1 + D.S - 1) / D.S;
     P.ntiles = D.topk + P.wtiles;
+    P.nparts = P.n > 0 ? (P.n + kSelPart - 1) / kSelPart : 1;
     size_t off = 0;
     auto take = [&](size_t bytes) {
         size_t at = off;
         off += (bytes + 255) & ~(size_t)255;
         return at;
     };
-    const size_t BG = (size_t)D.B * D.Hkv;
-    P.off_part = take(BG * P.nslices * D.G * 2 * sizeof(float));
-    P.off_list = take(BG * P.nslices * D.G * P.K1 * sizeof(uint64_t));
-    P.off_sel = take(BG * D.topk * sizeof(int));
+    P.off_scores = take((size_t)D.B * D.Hq * (P.n > 0 ? P.n : 1) * sizeof(float));
+    P.off_part = take((size_t)D.B * D.Hq * P.nslices * kScorePartsPerSliceHost * 2 * sizeof(float));
+    P.off_list = take((size_t)bg * P.nparts * D.topk * sizeof(uint64_t));
+    P.off_sel = take((size_t)bg * D.topk * sizeof(int));
     P.off_attn = take((size_t)D.B * D.Hq * P.ntiles * (D.d + 2) * sizeof(float));
+    P.off_count = take((size_t)bg * sizeof(unsigned int));
+    P.off_selcount = take((size_t)bg * sizeof(unsigned int));
     P.total = off;
     return P;
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kScoreThreads)
-decode_score_kernel(Dims D, DecodePlan P, const T *__restrict__ q_hat, const T *__restrict__ k_sum,
-                    const float *__restrict__ b_sum, float *__restrict__ part, uint64_t *__restrict__ lists) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-    const int d = D.d, G = D.G;
-    const int c0 = s * P.per;
-    const int c1 = min(P.n, c0 + P.per);
-    const int R = max(0, c1 - c0);
-    const int rpad = next_pow2(max(R, 1));
-    uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);  // [rpad]
-    float *qs = reinterpret_cast<float *>(keys + rpad);        // [G][d]
-    __shared__ float red[kScoreThreads / 32][2];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+// ---------------------------------------------------------------------------- 1. score
 
-    for (int e = threadIdx.x; e < G * d; e += blockDim.x) {
-        const int hh = e / d, t = e % d;
-        qs[e] = to_f(q_hat[((size_t)b * D.Hq + g * G + hh) * d + t]) * D.tau;
+// Persistent, warp-specialised: one CTA per SM; lane 0 of the last warp keeps a ring of kStages slice
+// copies in flight (one TMA bulk copy of P.per summary rows each: 32 KiB in bf16, 64 KiB in fp32).
+// kWarpsPerSlot consumer warps share each ring slot, one row per lane. A unit is (b, h, slice); each
+// consumer warp writes a partial (max, sum exp) of its rows, so a slice has kWarpsPerSlot partials.
+template <typename T>
+struct ScoreCfg {
+    static constexpr int kStages = sizeof(T) == 2 ? 6 : 3;
+    static constexpr int kWarpsPerSlot = 4;
+    static constexpr int kConsumers = kStages * kWarpsPerSlot;
+    static constexpr int kThreads = (kConsumers + 1) * 32;
+    static constexpr int kQFloats = 16 * 12 + 32;  // per-warp q staging (padded chunks)
+};
+
+template <typename T>
+__global__ void __launch_bounds__(ScoreCfg<T>::kThreads)
+decode_score_kernel(Dims D, DecodePlan P, const T *__restrict__ q_hat, const T *__restrict__ k_sum,
+                    const float *__restrict__ b_sum, float *__restrict__ scores, float *__restrict__ part) {
+    using C = ScoreCfg<T>;
+    constexpr int NS = C::kStages, WPS = C::kWarpsPerSlot;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t full[NS], empty[NS];
+    const int d = D.d;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const size_t slot_bytes = (size_t)P.per * d * sizeof(T);
+    const int units = D.B * D.Hq * P.nslices;
+    if (tid == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], WPS);
+        }
+        fence_mbar_init();
     }
     __syncthreads();
-
-    const int lanes_per_row = d / 8;
-    const int rows_per_warp = 32 / lanes_per_row;
-    const int sub = lane / lanes_per_row, sl = lane % lanes_per_row;
-    const size_t bg = (size_t)b * D.Hkv + g;
-    for (int hh = 0; hh < G; ++hh) {
-        const int h = g * G + hh;
-        const T *ksh = k_sum + ((size_t)b * D.Hq + h) * D.Nc * d;
-        const float *bsh = b_sum + ((size_t)b * D.Hq + h) * D.Nc;
-        const float *qq = qs + hh * d + sl * 8;
-        constexpr int U = 4;
-        for (int r0 = warp * rows_per_warp * U; r0 < rpad; r0 += nwarps * rows_per_warp * U) {
-            float f[U][8];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int r = r0 + u * rows_per_warp + sub;
-                if (r < R) load8(ksh + (size_t)(c0 + r) * d + sl * 8, f[u]);
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int r = r0 + u * rows_per_warp + sub;
-                float part_dot = 0.f;
-                if (r < R) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) part_dot = fmaf(f[u][e], qq[e], part_dot);
+    if (warp == C::kConsumers) {
+        if (lane == 0) {
+            int k = 0;
+            for (int u = blockIdx.x; u < units; u += gridDim.x, ++k) {
+                const int slot = k % NS, round = k / NS;
+                if (round > 0 && !mbar_wait_bounded(&empty[slot], (round - 1) & 1)) {
+                    atomicOr(&g_decode_errors, 1u);
+                    break;
                 }
-                for (int o = lanes_per_row / 2; o > 0; o >>= 1) part_dot += __shfl_xor_sync(0xffffffffu, part_dot, o);
-                if (sl == 0 && r < rpad)
-                    keys[r] = (r < R) ? desc_value_key(part_dot + bsh[c0 + r], (uint32_t)(c0 + r)) : ~0ull;
+                const int sl = u % P.nslices;
+                const size_t hrow = (size_t)(u / P.nslices);
+                const int c0 = sl * P.per;
+                const int R = min(P.n, c0 + P.per) - c0;
+                const uint32_t bytes = (uint32_t)(R * d * sizeof(T));
+                mbar_arrive_expect_tx(&full[slot], bytes);
+                bulk_g2s(smem_raw + slot * slot_bytes, k_sum + (hrow * D.Nc + c0) * d, bytes, &full[slot]);
             }
         }
-        __syncthreads();
-        // Partial (max, sum exp) of this head's slice.
-        float mx = -INFINITY;
-        for (int r = threadIdx.x; r < R; r += blockDim.x) mx = fmaxf(mx, desc_key_value(keys[r]));
-        mx = warp_max(mx);
-        if (lane == 0) red[warp][0] = mx;
-        __syncthreads();
-        mx = -INFINITY;
-        for (int w = 0; w < nwarps; ++w) mx = fmaxf(mx, red[w][0]);
-        float z = 0.f;
-        for (int r = threadIdx.x; r < R; r += blockDim.x) z += __expf(desc_key_value(keys[r]) - mx);
-        z = warp_sum(z);
-        if (lane == 0) red[warp][1] = z;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            float zz = 0.f;
-            for (int w = 0; w < nwarps; ++w) zz += red[w][1];
-            float *pp = part + ((bg * P.nslices + s) * G + hh) * 2;
-            pp[0] = mx;
-            pp[1] = zz;
+        return;
+    }
+    // Consumer warp: ring slot `slot`, quarter `qw` of the slot's rows (rows qw*32 + lane + 128*i).
+    // Rows are read in 16-byte chunks in a lane-rotated order (chunk (k + lane) mod NCH at step k), so
+    // the 8 lanes of a shared-memory phase hit 8 distinct bank groups; q^ (tau folded) is staged per
+    // warp as fp32 chunks with a padded stride.
+    constexpr int EC = 16 / sizeof(T);       // elements per 16-byte chunk
+    constexpr int QS = (EC == 8) ? 12 : EC;  // padded fp32 stride of one q chunk
+    const int NCH = d / EC;
+    const int slot = warp / WPS, qw = warp % WPS;
+    const T *rows = reinterpret_cast<const T *>(smem_raw + slot * slot_bytes);
+    float *qsm = reinterpret_cast<float *>(smem_raw + NS * slot_bytes) + warp * C::kQFloats;
+    constexpr int RPL = kSliceElems / 64 / (32 * WPS);  // rows per lane at d 64 (upper bound): 2
+    float nq[4], nb[RPL];
+    auto rows_of = [&](int u, int &c0, int &R, size_t &hrow, int &sl) {
+        sl = u % P.nslices;
+        hrow = (size_t)(u / P.nslices);
+        c0 = sl * P.per;
+        R = min(P.n, c0 + P.per) - c0;
+    };
+    auto prefetch = [&](int u) {
+        if (u >= units) return;
+        int c0, R, sl;
+        size_t hrow;
+        rows_of(u, c0, R, hrow, sl);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) nq[i] = (lane + 32 * i < d) ? to_f(q_hat[hrow * d + lane + 32 * i]) : 0.f;
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+            const int r = qw * 32 + lane + 32 * WPS * i;
+            nb[i] = (r < R) ? b_sum[hrow * D.Nc + c0 + r] : 0.f;
         }
-        block_bitonic_sort(keys, rpad);
-        uint64_t *lst = lists + ((bg * P.nslices + s) * G + hh) * P.K1;
-        for (int t = threadIdx.x; t < P.K1; t += blockDim.x) lst[t] = (t < R) ? keys[t] : ~0ull;
-        __syncthreads();
+    };
+    int k = slot;
+    prefetch(blockIdx.x + slot * gridDim.x);
+    for (int u = blockIdx.x + slot * gridDim.x; u < units; u += NS * gridDim.x, k += NS) {
+        const int round = k / NS;
+        int c0, R, sl;
+        size_t hrow;
+        rows_of(u, c0, R, hrow, sl);
+        float bcur[RPL];
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) bcur[i] = nb[i];
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int e = lane + 32 * i;
+            if (e < d) qsm[(e / EC) * QS + (e % EC)] = nq[i] * D.tau;
+        }
+        __syncwarp();
+        prefetch(u + NS * gridDim.x);  // overlaps this unit's wait and compute
+        if (!mbar_wait_bounded(&full[slot], round & 1)) {
+            if (lane == 0) atomicOr(&g_decode_errors, 1u);
+            return;
+        }
+        float acc[RPL];
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) acc[i] = 0.f;
+#pragma unroll 4
+        for (int kk = 0; kk < NCH; ++kk) {
+            const int ch = (kk + lane) & (NCH - 1);
+            float qv[EC];
+#pragma unroll
+            for (int e = 0; e < EC; e += 4) {
+                const float4 q4 = *reinterpret_cast<const float4 *>(qsm + ch * QS + e);
+                qv[e] = q4.x; qv[e + 1] = q4.y; qv[e + 2] = q4.z; qv[e + 3] = q4.w;
+            }
+#pragma unroll
+            for (int i = 0; i < RPL; ++i) {
+                const int r = qw * 32 + lane + 32 * WPS * i;
+                if (r < R) {
+                    float f[EC];
+                    if (EC == 8) {
+                        load8(reinterpret_cast<const __nv_bfloat16 *>(rows) + (size_t)r * d + ch * EC, f);
+                    } else {
+                        const float4 v4 = *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(rows) +
+                                                                            (size_t)r * d + ch * EC);
+                        f[0] = v4.x; f[1] = v4.y; f[2] = v4.z; f[3] = v4.w;
+                    }
+#pragma unroll
+                    for (int e = 0; e < EC; ++e) acc[i] = fmaf(f[e], qv[e], acc[i]);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);  // this warp is done with the slot
+        float m = -INFINITY, z = 0.f;
+        float *sch = scores + hrow * P.n + c0;
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+            const int r = qw * 32 + lane + 32 * WPS * i;
+            if (r < R) {
+                const float sc = acc[i] + bcur[i];
+                sch[r] = sc;
+                if (sc > m) {
+                    z = z * __expf(m - sc) + 1.f;
+                    m = sc;
+                } else {
+                    z += __expf(sc - m);
+                }
+            }
+        }
+        const float M = warp_max(m);
+        float Z = (m > -INFINITY) ? z * __expf(m - M) : 0.f;
+        Z = warp_sum(Z);
+        if (lane == 0) {
+            float *pp = part + ((hrow * P.nslices + sl) * kScorePartsPerSliceHost + qw) * 2;
+            pp[0] = M;
+            pp[1] = Z;
+        }
     }
 }
 
+// ---------------------------------------------------------------------------- 2. select
+
+// Ascending bitonic sort of 32*NPL 64-bit keys held in registers by one warp; element e of the
+// sequence is v[e % NPL] of lane e / NPL. No shared memory, no barriers.
+template <int NPL>
+__device__ __forceinline__ void warp_bitonic_sort(uint64_t (&v)[NPL]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int size = 2; size <= 32 * NPL; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            if (stride >= NPL) {
+                const int ls = stride / NPL;
+                const bool lower = (lane & ls) == 0;
+#pragma unroll
+                for (int i = 0; i < NPL; ++i) {
+                    const int e = lane * NPL + i;
+                    const bool up = (e & size) == 0;
+                    const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v[i], ls);
+                    const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v[i] >> 32), ls);
+                    const uint64_t p = ((uint64_t)hi << 32) | lo;
+                    const bool keep_min = (lower == up);
+                    v[i] = keep_min ? (v[i] < p ? v[i] : p) : (v[i] > p ? v[i] : p);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < NPL; ++i) {
+                    const int j = i ^ stride;
+                    if (j > i) {
+                        const int e = lane * NPL + i;
+                        const bool up = (e & size) == 0;
+                        if ((v[i] > v[j]) == up) {
+                            const uint64_t t = v[i];
+                            v[i] = v[j];
+                            v[j] = t;
+                        }
+                    }
+                }
+            }
+        }
+    }
+}
+
+// Grid (parts, Hkv, B): each CTA owns kSelPart candidates of one group. It folds the per-head score
+// partials into LSE_h, forms 64-bit keys (group score desc, chunk id asc; all distinct), keeps its
+// local top-k by a shared-memory bitonic sort and writes them to the workspace. The last CTA of the
+// group to finish (an atomic counter, no waiting) sorts the parts' lists and writes the group's top-k.
+// Exact: every member of the group's top-k is in its own part's top-k.
 __global__ void __launch_bounds__(kSelThreads)
-decode_select_kernel(Dims D, DecodePlan P, const float *__restrict__ part, const uint64_t *__restrict__ lists,
-                     int *__restrict__ sel, int *__restrict__ idx_out) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    const int g = blockIdx.x, b = blockIdx.y;
-    const int G = D.G, K = D.topk;
+decode_select_kernel(Dims D, DecodePlan P, const float *__restrict__ scores, const float *__restrict__ part,
+                     uint64_t *__restrict__ lists, unsigned int *__restrict__ counters, int *__restrict__ sel,
+                     int *__restrict__ idx_out) {
+    __shared__ float lse[64];
+    __shared__ __align__(8) uint64_t keys[kSelMerge];
+    __shared__ int s_last;
+    const int pidx = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int G = D.G, K = D.topk, n = P.n;
     const size_t bg = (size_t)b * D.Hkv + g;
-    const int E = P.nslices * G * P.K1;
-    const int epad = next_pow2(max(E, 1));
-    uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);  // [epad]
-    float *lse = reinterpret_cast<float *>(keys + epad);       // [G]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
     int *out = sel + bg * K;
     int *out2 = idx_out ? idx_out + bg * K : nullptr;
-    if (P.n == 0) {
-        for (int t = threadIdx.x; t < K; t += blockDim.x) {
+    if (n == 0) {
+        for (int t = tid; t < K; t += blockDim.x) {
             out[t] = -1;
             if (out2) out2[t] = -1;
         }
         return;
     }
-    for (int hh = threadIdx.x; hh < G; hh += blockDim.x) {
-        float M = -INFINITY;
-        for (int s = 0; s < P.nslices; ++s) M = fmaxf(M, part[((bg * P.nslices + s) * G + hh) * 2]);
-        float Z = 0.f;
-        for (int s = 0; s < P.nslices; ++s) {
-            const float *pp = part + ((bg * P.nslices + s) * G + hh) * 2;
-            if (pp[0] > -INFINITY) Z += pp[1] * __expf(pp[0] - M);
+    // Raw scores of this thread's candidates for the first kSelHeadsInFlight heads are loaded before
+    // the LSE fold, so both global round trips overlap.
+    const int c0 = pidx * kSelPart;
+    const float *sc0 = scores + ((size_t)b * D.Hq + g * G) * n;
+    constexpr int PER = kSelPart / kSelThreads;
+    float raw[kSelHeadsInFlight][PER];
+#pragma unroll
+    for (int hh = 0; hh < kSelHeadsInFlight; ++hh)
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int c = c0 + i * blockDim.x + tid;
+            raw[hh][i] = (hh < G && c < n) ? sc0[(size_t)hh * n + c] : -INFINITY;
         }
-        lse[hh] = M + logf(Z);
-    }
-    __syncthreads();
-    // Pass 1: order the entries by (chunk asc, normalised score desc).
-    for (int e = threadIdx.x; e < epad; e += blockDim.x) {
-        uint64_t key = ~0ull;
-        if (e < E) {
-            const uint64_t raw = lists[bg * (size_t)P.nslices * G * P.K1 + e];
-            if (raw != ~0ull) {
-                const int hh = (e / P.K1) % G;
-                const float val = desc_key_value(raw) - lse[hh];
-                key = ((uint64_t)desc_key_index(raw) << 32) | (uint64_t)(~float_order_key(val));
+    for (int hh = warp; hh < G; hh += nwarps) {
+        // online merge of the head's partials: each lane folds its entries, then the warp folds lanes
+        const int np = P.nslices * kScorePartsPerSliceHost;
+        const float2 *ph = reinterpret_cast<const float2 *>(part + ((size_t)b * D.Hq + g * G + hh) * np * 2);
+        float M = -INFINITY, Z = 0.f;
+        for (int s0 = 0; s0 < np; s0 += 32 * 8) {
+            float2 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int si = s0 + u * 32 + lane;
+                v[u] = (si < np) ? ph[si] : make_float2(-INFINITY, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (v[u].x > M) {
+                    Z = Z * __expf(M - v[u].x) + v[u].y;
+                    M = v[u].x;
+                } else if (v[u].x > -INFINITY) {
+                    Z += v[u].y * __expf(v[u].x - M);
+                }
             }
         }
-        keys[e] = key;
-    }
-    block_bitonic_sort(keys, epad);
-    // Keep the first (largest) entry of each chunk, re-keyed by (value desc, chunk asc).
-    uint64_t mine[16];
-    int cnt = 0;
-    for (int e = threadIdx.x; e < epad; e += blockDim.x) {
-        const uint64_t k0 = keys[e];
-        uint64_t nk = ~0ull;
-        if (k0 != ~0ull && (e == 0 || (keys[e - 1] >> 32) != (k0 >> 32))) {
-            const float val = float_from_order_key(~(uint32_t)k0);
-            nk = desc_value_key(val, (uint32_t)(k0 >> 32));
-        }
-        mine[cnt++] = nk;
+        const float MM = warp_max(M);
+        Z = (M > -INFINITY) ? Z * __expf(M - MM) : 0.f;
+        Z = warp_sum(Z);
+        if (lane == 0) lse[hh] = MM + logf(Z);
     }
     __syncthreads();
-    cnt = 0;
-    for (int e = threadIdx.x; e < epad; e += blockDim.x) keys[e] = mine[cnt++];
-    block_bitonic_sort(keys, epad);
-    const int kk = min(K, P.n);
-    for (int t = threadIdx.x; t < K; t += blockDim.x) {
+    float gv[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) gv[i] = -INFINITY;
+#pragma unroll
+    for (int hh = 0; hh < kSelHeadsInFlight; ++hh) {
+        if (hh < G) {
+            const float l = lse[hh];
+#pragma unroll
+            for (int i = 0; i < PER; ++i) gv[i] = fmaxf(gv[i], raw[hh][i] - l);
+        }
+    }
+    for (int hh = kSelHeadsInFlight; hh < G; ++hh) {  // groups wider than kSelHeadsInFlight heads
+        const float l = lse[hh];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int c = c0 + i * blockDim.x + tid;
+            if (c < n) gv[i] = fmaxf(gv[i], sc0[(size_t)hh * n + c] - l);
+        }
+    }
+    // Each warp sorts its 32*PER keys in registers and offers its best min(K, 32*PER) to shared memory.
+    uint64_t kv[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int c = c0 + i * blockDim.x + tid;
+        kv[i] = (c < n) ? desc_value_key(gv[i], (uint32_t)c) : ~0ull;
+    }
+    warp_bitonic_sort<PER>(kv);
+    const int KW = min(K, 32 * PER);  // survivors per warp
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int e = lane * PER + i;
+        if (e < KW) keys[warp * KW + e] = kv[i];
+    }
+    __syncthreads();
+    uint64_t *mine = lists + (bg * P.nparts + pidx) * K;
+    {
+        // Warp 0 sorts the nwarps*KW survivors (<= 256 = 32 x 8) and writes this part's top-K; more
+        // survivors (topk > 32) take the block-wide sort.
+        const int E1 = nwarps * KW;
+        if (E1 > 256) {
+            const int epad = next_pow2(E1);
+            for (int e = E1 + tid; e < epad; e += blockDim.x) keys[e] = ~0ull;
+            block_bitonic_sort(keys, epad);
+            for (int e = tid; e < K; e += blockDim.x) mine[e] = keys[e];
+        } else if (warp == 0) {
+            uint64_t w8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int e = lane * 8 + i;
+                w8[i] = (e < E1) ? keys[e] : ~0ull;
+            }
+            warp_bitonic_sort<8>(w8);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int e = lane * 8 + i;
+                if (e < K) mine[e] = w8[i];
+            }
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        s_last = (atomicAdd(&counters[bg], 1u) == (unsigned)(P.nparts - 1));
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const int E = P.nparts * K;
+    if (E <= 256) {
+        if (warp == 0) {
+            uint64_t w8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int e = lane * 8 + i;
+                w8[i] = (e < E) ? __ldcg(lists + bg * P.nparts * K + e) : ~0ull;
+            }
+            warp_bitonic_sort<8>(w8);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int e = lane * 8 + i;
+                if (e < K) keys[e] = w8[i];
+            }
+        }
+        __syncthreads();
+    } else {
+        const int epad = next_pow2(E);
+        for (int e = tid; e < epad; e += blockDim.x) keys[e] = (e < E) ? __ldcg(lists + bg * P.nparts * K + e) : ~0ull;
+        block_bitonic_sort(keys, epad);
+    }
+    const int kk = min(K, n);
+    for (int t = tid; t < K; t += blockDim.x) {
         if (t < kk) {
             const uint32_t me = desc_key_index(keys[t]);
             int rank = 0;
@@ -221,25 +452,34 @@ decode_select_kernel(Dims D, DecodePlan P, const float *__restrict__ part, const
     }
 }
 
+// ---------------------------------------------------------------------------- 3. attend (+ combine)
+
 template <typename T, int DPL>
 __global__ void __launch_bounds__(kAttnThreads)
-decode_attn_kernel(Dims D, DecodePlan P, const T *__restrict__ q, const T *__restrict__ q_hat,
-                   const T *__restrict__ kc, const T *__restrict__ vc, const T *__restrict__ k_sum,
-                   const float *__restrict__ b_sum, const int *__restrict__ sel, float *__restrict__ partial) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
+decode_attn_kernel(Dims D, DecodePlan P, const T *__restrict__ q, const T *__restrict__ kc,
+                   const T *__restrict__ vc, const float *__restrict__ scores, const int *__restrict__ sel,
+                   float *__restrict__ partial, unsigned int *__restrict__ counters, T *__restrict__ out,
+                   float *__restrict__ lse) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int s_last;
     const int t = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int d = D.d, S = D.S, G = D.G;
-    const int ld = d + 1;
-    float *ks = reinterpret_cast<float *>(smem_raw);  // [S][d+1]
-    float *vs = ks + S * ld;                          // [S][d]
-    float *qs = vs + S * d;                           // [G][d]
-    float *ls = qs + G * d;                           // [warps][S]
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nwarps = blockDim.x >> 5;
     const size_t bg = (size_t)b * D.Hkv + g;
     const int pos = D.L - 1;
     const int l = window_left(pos, D.W, S);
+    T *ks = reinterpret_cast<T *>(smem_raw);                    // [S][d]
+    T *vs = ks + (size_t)S * d;                                 // [S][d]
+    float *ws = reinterpret_cast<float *>(vs + (size_t)S * d);  // [G][S] logits, then weights
+    constexpr int EC = 16 / sizeof(T);        // elements per 16-byte chunk
+    constexpr int QS = (EC == 8) ? 12 : EC;   // padded fp32 stride of one q chunk
+    const int NCH = d / EC;
+    float *qs = ws + ((G * S + 3) & ~3);      // [G][NCH][QS] q chunks, tau folded (16-byte aligned)
+    float *shat = qs + G * NCH * QS;          // [G] retrieval scores of the tile's chunk
+    float *half = shat + ((G + 3) & ~3);      // [2G][32][DPL] value-product halves
 
-    int c = -1, j0 = 0, jn = 0;  // tile tokens [j0, j0 + jn)
+    int c = -1, j0 = 0, jn = 0;
     if (t < D.topk) {
         c = sel[bg * D.topk + t];
         if (c >= 0) { j0 = c * S; jn = S; }
@@ -247,131 +487,208 @@ decode_attn_kernel(Dims D, DecodePlan P, const T *__restrict__ q, const T *__res
         j0 = l + (t - D.topk) * S;
         jn = min(S, pos + 1 - j0);
     }
-    if (jn <= 0) {
+    bool ok = true;
+    if (jn > 0) {
+        const uint32_t bytes = (uint32_t)(jn * d * sizeof(T));
+        if (tid == 0) {
+            mbar_init(&bar, 1);
+            fence_mbar_init();
+        }
+        __syncthreads();
+        if (tid == 0) {
+            mbar_arrive_expect_tx(&bar, 2 * bytes);
+            bulk_g2s(ks, kc + (bg * D.L + j0) * d, bytes, &bar);
+            bulk_g2s(vs, vc + (bg * D.L + j0) * d, bytes, &bar);
+        }
+        for (int e = tid; e < G * d; e += blockDim.x) {
+            const int hh = e / d, x = e % d;
+            qs[(hh * NCH + x / EC) * QS + x % EC] = to_f(q[((size_t)b * D.Hq + g * G) * d + e]) * D.tau;
+        }
+        if (c >= 0)  // the chunk's retrieval score per head, fetched while the tile is in flight
+            for (int hh = tid; hh < G; hh += blockDim.x) shat[hh] = scores[((size_t)b * D.Hq + g * G + hh) * P.n + c];
+        ok = mbar_wait_bounded(&bar, 0);
+        if (!ok && tid == 0) atomicOr(&g_decode_errors, 1u);
+        __syncthreads();
+    }
+    if (jn > 0 && ok) {
+        // Logits: one (token j, head) item per thread; K chunks read in a token-rotated order so the 8
+        // lanes of a shared-memory phase hit distinct bank groups.
+        for (int e = tid; e < G * S; e += blockDim.x) {
+            const int j = e % S, hh = e / S;
+            float acc = -INFINITY;
+            if (j < jn) {
+                float acc2 = 0.f;  // second chain halves the dependent-FMA latency
+                acc = 0.f;
+                const float *qh = qs + hh * NCH * QS;
+#pragma unroll 4
+                for (int kk = 0; kk < NCH; ++kk) {
+                    const int ch = (kk + j) & (NCH - 1);
+                    float f[EC];
+                    if (EC == 8) {
+                        load8(reinterpret_cast<const __nv_bfloat16 *>(ks) + (size_t)j * d + ch * EC, f);
+                    } else {
+                        const float4 v4 = *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(ks) +
+                                                                            (size_t)j * d + ch * EC);
+                        f[0] = v4.x; f[1] = v4.y; f[2] = v4.z; f[3] = v4.w;
+                    }
+#pragma unroll
+                    for (int x = 0; x < EC; x += 4) {
+                        const float4 q4 = *reinterpret_cast<const float4 *>(qh + ch * QS + x);
+                        acc = fmaf(f[x], q4.x, acc);
+                        acc2 = fmaf(f[x + 1], q4.y, acc2);
+                        acc = fmaf(f[x + 2], q4.z, acc);
+                        acc2 = fmaf(f[x + 3], q4.w, acc2);
+                    }
+                }
+                acc += acc2;
+            }
+            ws[hh * S + j] = acc;
+        }
+        __syncthreads();
         for (int hh = warp; hh < G; hh += nwarps) {
+            float mx = -INFINITY;
+            for (int j = lane; j < S; j += 32) mx = fmaxf(mx, ws[hh * S + j]);
+            mx = warp_max(mx);
+            float z = 0.f;
+            for (int j = lane; j < S; j += 32) {
+                const float e = __expf(ws[hh * S + j] - mx);  // padding: exp(-inf) = 0
+                ws[hh * S + j] = e;
+                z += e;
+            }
+            z = warp_sum(z);
+            // Chunk tile: tokens carry exp(s_j - L_c + s^_c); relative to m = s^_c - log z their weights
+            // are exp(s_j - mx) and sum to z. Window tile: m = mx.
+            if (lane == 0) {
+                float *pp = partial + (((size_t)b * D.Hq + g * G + hh) * P.ntiles + t) * (d + 2);
+                pp[0] = (c >= 0) ? shat[hh] - logf(z) : mx;
+                pp[1] = z;
+            }
+        }
+        __syncthreads();
+        // Value product: (head, half of the tokens) per warp, lane owns DPL dims; halves meet in smem.
+        for (int wk = warp; wk < 2 * G; wk += nwarps) {
+            const int hh = wk >> 1, hf = wk & 1;
+            const int jb = hf * ((jn + 1) / 2), je = hf ? jn : (jn + 1) / 2;
+            float acc[DPL], acc2[DPL];
+#pragma unroll
+            for (int u = 0; u < DPL; ++u) { acc[u] = 0.f; acc2[u] = 0.f; }
+            int j = jb;
+            for (; j + 1 < je; j += 2) {
+                const float w0 = ws[hh * S + j], w1 = ws[hh * S + j + 1];
+#pragma unroll
+                for (int u = 0; u < DPL; ++u) {
+                    acc[u] = fmaf(w0, to_f(vs[(size_t)j * d + lane * DPL + u]), acc[u]);
+                    acc2[u] = fmaf(w1, to_f(vs[(size_t)(j + 1) * d + lane * DPL + u]), acc2[u]);
+                }
+            }
+            if (j < je) {
+                const float w0 = ws[hh * S + j];
+#pragma unroll
+                for (int u = 0; u < DPL; ++u) acc[u] = fmaf(w0, to_f(vs[(size_t)j * d + lane * DPL + u]), acc[u]);
+            }
+#pragma unroll
+            for (int u = 0; u < DPL; ++u) half[(wk * 32 + lane) * DPL + u] = acc[u] + acc2[u];
+        }
+        __syncthreads();
+        for (int e = tid; e < G * d; e += blockDim.x) {
+            const int hh = e / d, x = e % d;
+            const int ln = x / DPL, u = x % DPL;
+            partial[(((size_t)b * D.Hq + g * G + hh) * P.ntiles + t) * (d + 2) + 2 + x] =
+                half[((2 * hh) * 32 + ln) * DPL + u] + half[((2 * hh + 1) * 32 + ln) * DPL + u];
+        }
+    } else {
+        for (int hh = tid; hh < G; hh += blockDim.x) {
             float *pp = partial + (((size_t)b * D.Hq + g * G + hh) * P.ntiles + t) * (d + 2);
-            if (lane == 0) { pp[0] = -INFINITY; pp[1] = 0.f; }
+            pp[0] = -INFINITY;
+            pp[1] = 0.f;
         }
-        return;
     }
-    const T *kb = kc + (bg * D.L + j0) * d;
-    const T *vb = vc + (bg * D.L + j0) * d;
-    for (int e = threadIdx.x * 8; e < jn * d; e += blockDim.x * 8) {
-        float f[8];
-        load8(kb + e, f);
-        const int j = e / d, tt = e % d;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) ks[j * ld + tt + u] = f[u];
-        load8(vb + e, f);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) vs[e + u] = f[u];
-    }
-    for (int e = threadIdx.x; e < G * d; e += blockDim.x)
-        qs[e] = to_f(q[((size_t)b * D.Hq + g * G) * d + e]) * D.tau;
+    // The last tile of this (b, group) to finish merges all tiles' partials (no CTA waits on another).
     __syncthreads();
-
-    float *lw = ls + warp * S;
+    if (tid == 0) {
+        __threadfence();
+        s_last = (atomicAdd(&counters[bg], 1u) == (unsigned)(P.ntiles - 1));
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
     for (int hh = warp; hh < G; hh += nwarps) {
-        const int h = g * G + hh;
-        const float *qq = qs + hh * d;
-        float mx = -INFINITY;
-        for (int j = lane; j < jn; j += 32) {
-            const float *kj = ks + j * ld;
-            float s = 0.f;
-            for (int u = 0; u < d; ++u) s = fmaf(qq[u], kj[u], s);
-            lw[j] = s;
-            mx = fmaxf(mx, s);
+        const size_t bh = (size_t)b * D.Hq + g * G + hh;
+        const float *ph = partial + bh * P.ntiles * (d + 2);
+        float M = -INFINITY;
+        for (int u = lane; u < P.ntiles; u += 32) M = fmaxf(M, __ldcg(ph + (size_t)u * (d + 2)));
+        M = warp_max(M);
+        float Z = 0.f;
+        for (int u = lane; u < P.ntiles; u += 32) {
+            const float mu = __ldcg(ph + (size_t)u * (d + 2));
+            if (mu > -INFINITY) Z += __ldcg(ph + (size_t)u * (d + 2) + 1) * __expf(mu - M);
         }
-        mx = warp_max(mx);
-        float offset = 0.f;
-        if (c >= 0) {
-            float zc = 0.f;
-            for (int j = lane; j < jn; j += 32) zc += __expf(lw[j] - mx);
-            zc = warp_sum(zc);
-            const size_t srow = ((size_t)b * D.Hq + h) * D.Nc + c;
-            float sh = 0.f;
+        Z = warp_sum(Z);
+        // tile weights exp(m_t - M), held by lane t % 32 (two registers for up to 64 tiles)
+        float r0 = 0.f, r1 = 0.f;
+        if (lane < P.ntiles) {
+            const float mu = __ldcg(ph + (size_t)lane * (d + 2));
+            r0 = (mu > -INFINITY) ? __expf(mu - M) : 0.f;
+        }
+        if (lane + 32 < P.ntiles) {
+            const float mu = __ldcg(ph + (size_t)(lane + 32) * (d + 2));
+            r1 = (mu > -INFINITY) ? __expf(mu - M) : 0.f;
+        }
+        float acc[DPL];
 #pragma unroll
-            for (int u = 0; u < DPL; ++u)
-                sh = fmaf(to_f(q_hat[((size_t)b * D.Hq + h) * d + lane + 32 * u]), to_f(k_sum[srow * d + lane + 32 * u]),
-                          sh);
-            sh = warp_sum(sh) * D.tau + b_sum[srow];
-            offset = sh - (mx + logf(zc));
+        for (int u = 0; u < DPL; ++u) acc[u] = 0.f;
+#pragma unroll 8
+        for (int tt = 0; tt < P.ntiles; ++tt) {
+            const float r = __shfl_sync(0xffffffffu, tt < 32 ? r0 : r1, tt & 31);
+#pragma unroll
+            for (int u = 0; u < DPL; ++u) acc[u] = fmaf(__ldcg(ph + (size_t)tt * (d + 2) + 2 + lane * DPL + u), r, acc[u]);
         }
-        const float m = mx + offset;
-        float z = 0.f;
-        __syncwarp();
-        for (int j = lane; j < jn; j += 32) {
-            const float w = __expf(lw[j] + offset - m);
-            lw[j] = w;
-            z += w;
-        }
-        z = warp_sum(z);
-        __syncwarp();
-        float *pp = partial + (((size_t)b * D.Hq + h) * P.ntiles + t) * (d + 2);
-        for (int u = lane; u < d; u += 32) {
-            float acc = 0.f;
-            for (int j = 0; j < jn; ++j) acc = fmaf(lw[j], vs[j * d + u], acc);
-            pp[2 + u] = acc;
-        }
-        if (lane == 0) { pp[0] = m; pp[1] = z; }
-        __syncwarp();
+        const float inv = 1.f / Z;
+#pragma unroll
+        for (int u = 0; u < DPL; ++u) out[bh * d + lane * DPL + u] = from_f<T>(acc[u] * inv);
+        if (lane == 0) lse[bh] = M + logf(Z);
     }
 }
 
-template <typename T>
-__global__ void decode_combine_kernel(Dims D, DecodePlan P, const float *__restrict__ partial, T *__restrict__ out,
-                                      float *__restrict__ lse) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.x * (blockDim.x >> 5) + warp;
-    if (bh >= D.B * D.Hq) return;
-    const int d = D.d;
-    const float *pp = partial + (size_t)bh * P.ntiles * (d + 2);
-    float M = -INFINITY;
-    for (int t = 0; t < P.ntiles; ++t) M = fmaxf(M, pp[t * (d + 2)]);
-    float Z = 0.f;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int t = 0; t < P.ntiles; ++t) {
-        const float m = pp[t * (d + 2)];
-        if (!(m > -INFINITY)) continue;
-        const float r = __expf(m - M);
-        Z = fmaf(pp[t * (d + 2) + 1], r, Z);
-        for (int u = 0; u < d / 32; ++u) acc[u] = fmaf(pp[t * (d + 2) + 2 + lane + 32 * u], r, acc[u]);
-    }
-    const float inv = 1.f / Z;
-    for (int u = 0; u < d / 32; ++u) out[(size_t)bh * d + lane + 32 * u] = from_f<T>(acc[u] * inv);
-    if (lane == 0) lse[bh] = M + logf(Z);
-}
-
-template <typename T>
+template <typename T, int DPL>
 cudaError_t launch_t(const Dims &D, const void *q, const void *q_hat, const void *k_cache, const void *v_cache,
                      const void *k_sum, const float *b_sum, void *out, float *lse, int *idx_out, void *ws,
                      cudaStream_t stream) {
     const DecodePlan P = make_plan(D);
     unsigned char *w = (unsigned char *)ws;
+    float *scores = (float *)(w + P.off_scores);
     float *part = (float *)(w + P.off_part);
     uint64_t *lists = (uint64_t *)(w + P.off_list);
     int *sel = (int *)(w + P.off_sel);
     float *partial = (float *)(w + P.off_attn);
+    unsigned int *counters = (unsigned int *)(w + P.off_count);
+    // Both counter arrays (attention, selection) are adjacent: clear them in one call.
+    cudaError_t e = cudaMemsetAsync(counters, 0, P.total - P.off_count, stream);
+    if (e != cudaSuccess) return e;
     if (P.n > 0) {
-        const size_t smem1 = (size_t)next_pow2(max(P.per, 1)) * 8 + (size_t)D.G * D.d * 4;
+        using C = ScoreCfg<T>;
+        static_assert(C::kWarpsPerSlot == kScorePartsPerSliceHost, "one partial per consumer warp of a slot");
+        const size_t smem1 = (size_t)C::kStages * P.per * D.d * sizeof(T) +
+                             (size_t)C::kConsumers * C::kQFloats * sizeof(float);
         auto k1 = decode_score_kernel<T>;
         cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
-        k1<<<dim3(P.nslices, D.Hkv, D.B), kScoreThreads, smem1, stream>>>(D, P, (const T *)q_hat, (const T *)k_sum,
-                                                                           b_sum, part, lists);
+        const int units = D.B * D.Hq * P.nslices;
+        const int sms = num_sms();
+        const int grid = units < sms ? units : sms;
+        k1<<<grid, ScoreCfg<T>::kThreads, smem1, stream>>>(D, P, (const T *)q_hat, (const T *)k_sum, b_sum, scores,
+                                                           part);
     }
-    const int E = P.nslices * D.G * P.K1;
-    const size_t smem2 = (size_t)next_pow2(max(E, 1)) * 8 + (size_t)D.G * 4 + 16;
-    cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
-    decode_select_kernel<<<dim3(D.Hkv, D.B), kSelThreads, smem2, stream>>>(D, P, part, lists, sel, idx_out);
-    const size_t smem3 = sizeof(float) * ((size_t)D.S * (D.d + 1) + (size_t)D.S * D.d + (size_t)D.G * D.d +
-                                          (size_t)(kAttnThreads / 32) * D.S);
-    auto k3 = (D.d == 128) ? decode_attn_kernel<T, 4> : decode_attn_kernel<T, 2>;
-    cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3);
-    k3<<<dim3(P.ntiles, D.Hkv, D.B), kAttnThreads, smem3, stream>>>(D, P, (const T *)q, (const T *)q_hat,
-                                                                     (const T *)k_cache, (const T *)v_cache,
-                                                                     (const T *)k_sum, b_sum, sel, partial);
-    const int rows = D.B * D.Hq;
-    decode_combine_kernel<T><<<(rows + 3) / 4, 128, 0, stream>>>(D, P, partial, (T *)out, lse);
+    unsigned int *selcount = (unsigned int *)(w + P.off_selcount);
+    decode_select_kernel<<<dim3(P.nparts, D.Hkv, D.B), kSelThreads, 0, stream>>>(D, P, scores, part, lists, selcount,
+                                                                                 sel, idx_out);
+    const size_t smem3 = 2 * (size_t)D.S * D.d * sizeof(T) +
+                         sizeof(float) * ((size_t)D.G * D.S + 4 + (size_t)D.G * D.d * 3 / 2 + D.G + 4 +
+                                          2 * (size_t)D.G * D.d);
+    auto k3 = decode_attn_kernel<T, DPL>;
+    if (smem3 > 48 * 1024) cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3);
+    k3<<<dim3(P.ntiles, D.Hkv, D.B), kAttnThreads, smem3, stream>>>(D, P, (const T *)q, (const T *)k_cache,
+                                                                     (const T *)v_cache, scores, sel, partial,
+                                                                     counters, (T *)out, lse);
     return cudaGetLastError();
 }
 
@@ -380,16 +697,34 @@ cudaError_t launch_t(const Dims &D, const void *q, const void *q_hat, const void
 size_t decode_workspace_bytes(const Dims &D) { return make_plan(D).total; }
 
 bool decode_supported(const Dims &D) {
+    // The attention tile (K and V of one chunk plus the per-head rows) must fit in shared memory.
+    const size_t el = 4;  // worst case fp32
+    const size_t smem3 = 2 * (size_t)D.S * D.d * el + 4 * ((size_t)D.G * D.S + 4 + (size_t)D.G * D.d * 3 / 2 + D.G + 4 + 2 * (size_t)D.G * D.d);
     const DecodePlan P = make_plan(D);
-    return P.per <= kMaxSliceChunks && P.nslices * D.G * P.K1 <= 2 * kMaxListEntries;
+    return D.G <= 64 && D.topk + (D.W + 2 * D.S) / D.S <= 64 && next_pow2(P.nparts * D.topk) <= kSelMerge &&
+           smem3 <= 200 * 1024;
+}
+
+unsigned int decode_error_flags(bool clear) {
+    unsigned int v = 0;
+    cudaMemcpyFromSymbol(&v, g_decode_errors, sizeof(v));
+    if (clear && v) {
+        const unsigned int zero = 0;
+        cudaMemcpyToSymbol(g_decode_errors, &zero, sizeof(zero));
+    }
+    return v;
 }
 
 cudaError_t launch_decode(const Dims &D, int dtype, const void *q, const void *q_hat, const void *k_cache,
                           const void *v_cache, const void *k_sum, const float *b_sum, void *out, float *lse,
                           int *idx_out, void *ws, cudaStream_t stream) {
-    if (dtype == HILS_BF16)
-        return launch_t<__nv_bfloat16>(D, q, q_hat, k_cache, v_cache, k_sum, b_sum, out, lse, idx_out, ws, stream);
-    return launch_t<float>(D, q, q_hat, k_cache, v_cache, k_sum, b_sum, out, lse, idx_out, ws, stream);
+    if (dtype == HILS_BF16) {
+        if (D.d == 128)
+            return launch_t<__nv_bfloat16, 4>(D, q, q_hat, k_cache, v_cache, k_sum, b_sum, out, lse, idx_out, ws, stream);
+        return launch_t<__nv_bfloat16, 2>(D, q, q_hat, k_cache, v_cache, k_sum, b_sum, out, lse, idx_out, ws, stream);
+    }
+    if (D.d == 128) return launch_t<float, 4>(D, q, q_hat, k_cache, v_cache, k_sum, b_sum, out, lse, idx_out, ws, stream);
+    return launch_t<float, 2>(D, q, q_hat, k_cache, v_cache, k_sum, b_sum, out, lse, idx_out, ws, stream);
 }
 
 }  // namespace hils

@@ -89,6 +89,13 @@ hils_status check_ws(const char *fn, void *ws, size_t have, size_t need) {
 // Lets other translation units of the library set the thread-local message of hils_last_error().
 void record_error(const char *msg) { g_last_error = msg; }
 
+hils_status check_device_errors() {
+    if (decode_error_flags(true) != 0)
+        return fail(HILS_ERR_TIMEOUT, "hils_check: a decode tile's bulk copy did not complete within its wait "
+                    "budget; that call's output is invalid");
+    return HILS_OK;
+}
+
 }  // namespace hils
 
 using namespace hils;

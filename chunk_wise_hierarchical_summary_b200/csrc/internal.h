@@ -25,6 +25,9 @@ cudaError_t launch_decode(const Dims &D, int dtype, const void *q, const void *q
                           const void *v_cache, const void *k_sum, const float *b_sum, void *out, float *lse,
                           int *idx_out, void *ws, cudaStream_t stream);
 
+// Device-side error words (bit set when a bounded wait expired); reading with clear resets them.
+unsigned int decode_error_flags(bool clear);
+
 size_t bwd_workspace_bytes(const Dims &D);
 cudaError_t launch_attn_bwd(const Dims &D, int dtype, const void *q, const void *k, const void *v, const void *q_hat,
                             const void *q_land, const void *k_sum, const float *b_sum, const int *idx,
