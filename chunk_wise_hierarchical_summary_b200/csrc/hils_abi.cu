@@ -21,6 +21,10 @@ cudaError_t launch_attn_fwd_tc(const Dims &D, const void *q, const void *k, cons
                                cudaStream_t stream);
 size_t attn_fwd_tc_workspace(const Dims &D);
 hils_status check_device_errors();
+bool select_tc_supported(const Dims &D, int dtype);
+cudaError_t launch_select_tc(const Dims &D, const void *q_hat, const void *k_sum, const float *b_sum, int *idx,
+                             float *gap, cudaStream_t stream);
+unsigned int select_tc_error_flags(bool clear);
 
 namespace {
 
@@ -90,6 +94,9 @@ hils_status check_ws(const char *fn, void *ws, size_t have, size_t need) {
 void record_error(const char *msg) { g_last_error = msg; }
 
 hils_status check_device_errors() {
+    if (select_tc_error_flags(true) != 0)
+        return fail(HILS_ERR_TIMEOUT, "hils_check: a tensor-core selection tile's wait expired; that call's ids are "
+                    "invalid");
     if (decode_error_flags(true) != 0)
         return fail(HILS_ERR_TIMEOUT, "hils_check: a decode tile's bulk copy did not complete within its wait "
                     "budget; that call's output is invalid");
@@ -167,6 +174,8 @@ hils_status hils_select_topk(const hils_params *p, const void *q_hat, const void
                     fn, D.Nc, D.G);
     st = check_ws(fn, workspace, workspace_bytes, 0);
     if (st != HILS_OK) return st;
+    if (select_tc_supported(D, p->dtype))
+        return cuda_status(launch_select_tc(D, q_hat, k_sum, b_sum, idx, gap, (cudaStream_t)stream), fn);
     return cuda_status(launch_select_topk(D, p->dtype, q_hat, k_sum, b_sum, idx, gap, (cudaStream_t)stream), fn);
 }
 

@@ -1,0 +1,266 @@
+// Stage (b) on the tensor cores, prefill form: retrieval scores (Eq. 7) and GQA-shared top-k
+// ("Hierarchical Sparse Attention Done Right", Sec. 3 RQ1, Sec. 4 "GQA"), bf16, d = 128.
+//
+// CTA = (128 query rows, KV group g, batch b); 16 warps. For each head h of the group one thread
+// TMA-loads the q^ tile [128 x 128] and the summary tile k'_h [128 chunks x 128] (128-byte swizzle,
+// two stages) and issues 8 tcgen05.mma (M 128, N 128, K 16) into TMEM columns [128h, 128h+128):
+// D[i][c] = q^_i . k'_c. Then, with rows in TMEM lanes:
+//   phase 1  warp (quadrant, head): s^ = tau D + b', masked to the row's candidates; LSE_h per row.
+//   phase 2  warp (quadrant, column block of 32): g_c = max_h (s^_{h,c} - LSE_h) as 64-bit keys
+//            (score desc, chunk id asc); each thread keeps its block's best K1 in a sorted register list.
+//   phase 3  one thread per row merges the four lists: top-k ids (ascending) and the gap.
+// Rows whose candidates exceed 128 chunks use the general kernel (select.cu).
+#include "internal.h"
+#include "tcgen05.cuh"
+
+namespace hils {
+
+bool make_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint64_t ld,
+                       uint32_t box_rows);
+
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kRows = 128;
+constexpr int kStageBytes = 65536;  // q^ tile (32 KiB) + k' tile (32 KiB)
+
+__device__ unsigned int g_select_tc_errors = 0;
+
+template <int K1MAX>
+__global__ void __launch_bounds__(kThreads, 1)
+select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, Dims D,
+                 const float *__restrict__ b_sum, int *__restrict__ idx, float *__restrict__ gap) {
+    extern __shared__ unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t tma_bar[2], mma_bar[2], done_bar;
+    __shared__ uint32_t s_tmem;
+    __shared__ float bs[4][kRows];
+    __shared__ float lse[4][kRows];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int i0 = blockIdx.x * kRows, g = blockIdx.y, b = blockIdx.z;
+    const int G = D.G, K = D.topk;
+    unsigned char *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);  // 1024-byte aligned
+    const uint32_t ncols = G == 1 ? 128 : (G == 2 ? 256 : 512);
+
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, ncols);
+        tmem_relinquish();
+    }
+    if (tid == 32) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tma_bar[i], 1);
+            mbar_init(&mma_bar[i], 1);
+        }
+        mbar_init(&done_bar, 1);
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            auto load = [&](int hh, int st) {
+                unsigned char *A = base + st * kStageBytes, *Bt = A + 32768;
+                const int hrow = b * D.Hq + g * G + hh;
+                mbar_arrive_expect_tx(&tma_bar[st], kStageBytes);
+                tma_load_2d(A, &qmap, 0, hrow * D.T + i0, &tma_bar[st]);
+                tma_load_2d(A + 16384, &qmap, 64, hrow * D.T + i0, &tma_bar[st]);
+                tma_load_2d(Bt, &kmap, 0, hrow * D.Nc, &tma_bar[st]);
+                tma_load_2d(Bt + 16384, &kmap, 64, hrow * D.Nc, &tma_bar[st]);
+            };
+            bool ok = true;
+            for (int hh = 0; hh < G && hh < 2; ++hh) load(hh, hh);
+            const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+            for (int hh = 0; hh < G && ok; ++hh) {
+                const int st = hh & 1;
+                if (!mbar_wait_bounded(&tma_bar[st], (hh >> 1) & 1)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t A = smem_u32(base + st * kStageBytes), Bt = A + 32768;
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    umma_bf16(tmem + hh * 128, sdesc_sw128(A + off, 16, 1024), sdesc_sw128(Bt + off, 16, 1024), idesc,
+                              ks > 0);
+                }
+                umma_commit(&mma_bar[st]);
+                if (hh + 2 < G) {
+                    if (!mbar_wait_bounded(&mma_bar[st], (hh >> 1) & 1)) { ok = false; break; }
+                    load(hh + 2, st);
+                }
+            }
+            if (!ok) atomicOr(&g_select_tc_errors, 1u);
+            umma_commit(&done_bar);  // arrives once every MMA issued above has completed
+        }
+        __syncwarp();
+    }
+    // b' of the group's heads for chunks [0, 128), -inf beyond the summaries.
+    for (int e = tid; e < 4 * kRows; e += blockDim.x) {
+        const int hh = e / kRows, c = e % kRows;
+        bs[hh][c] = (hh < G && c < D.Nc) ? b_sum[((size_t)b * D.Hq + g * G + hh) * D.Nc + c] : 0.f;
+    }
+    const bool ok = mbar_wait_bounded(&done_bar, 0);
+    tc_fence_after();
+    __syncthreads();
+    const int q = warp & 3, j = warp >> 2;
+    const int r = 32 * q + lane;  // tile row = TMEM lane
+    const int i = i0 + r;
+    const int n_r = (i < D.T) ? window_left(D.q_pos0 + i, D.W, D.S) / D.S : 0;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+
+    // Phase 1: per-head log-partition over the row's candidates.
+    if (j < G) {
+        const int hh = j;
+        float m = -INFINITY, z = 0.f;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            float v[32];
+            tmem_ld32(lane_base + hh * 128 + 32 * t, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int c = 32 * t + e;
+                if (c < n_r) {
+                    const float sc = fmaf(D.tau, v[e], bs[hh][c]);
+                    if (sc > m) {
+                        z = z * __expf(m - sc) + 1.f;
+                        m = sc;
+                    } else {
+                        z += __expf(sc - m);
+                    }
+                }
+            }
+        }
+        lse[hh][r] = (n_r > 0) ? m + logf(z) : 0.f;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // Phase 2: group scores of column block j, best K1MAX per row kept sorted in registers.
+    uint64_t top[K1MAX];
+#pragma unroll
+    for (int t = 0; t < K1MAX; ++t) top[t] = ~0ull;
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+        const int cb = 32 * j + 16 * half;  // first column of this 16-wide piece
+        float gv[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) gv[e] = -INFINITY;
+        for (int hh = 0; hh < G; ++hh) {
+            float v[16];
+            tmem_ld16(lane_base + hh * 128 + cb, v);
+            tmem_wait_ld();
+            const float l = lse[hh][r];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) gv[e] = fmaxf(gv[e], fmaf(D.tau, v[e], bs[hh][cb + e]) - l);
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int c = cb + e;
+            if (c < n_r) {
+                uint64_t x = desc_value_key(gv[e], (uint32_t)c);
+                if (x < top[K1MAX - 1]) {
+#pragma unroll
+                    for (int t = 0; t < K1MAX; ++t) {
+                        if (x < top[t]) {
+                            const uint64_t y = top[t];
+                            top[t] = x;
+                            x = y;
+                        }
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();  // every TMEM read done; operand tiles are dead: reuse them for the lists
+    uint64_t *lists = reinterpret_cast<uint64_t *>(base);  // [128 rows][4 blocks][K1MAX]
+#pragma unroll
+    for (int t = 0; t < K1MAX; ++t) lists[((size_t)r * 4 + j) * K1MAX + t] = top[t];
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, ncols);
+    }
+
+    // Phase 3: merge the four sorted lists of a row.
+    if (tid < kRows) {
+        const int rr = tid, ii = i0 + rr;
+        if (ii < D.T) {
+            const int nn = window_left(D.q_pos0 + ii, D.W, D.S) / D.S;
+            const uint64_t *L = lists + (size_t)rr * 4 * K1MAX;
+            int p0 = 0, p1 = 0, p2 = 0, p3 = 0;
+            const int need = min(K + 1, nn);
+            uint32_t ids[K1MAX];
+            float vk = 0.f, vk1 = 0.f;
+            for (int t = 0; t < need; ++t) {
+                const uint64_t a0 = p0 < K1MAX ? L[p0] : ~0ull, a1 = p1 < K1MAX ? L[K1MAX + p1] : ~0ull;
+                const uint64_t a2 = p2 < K1MAX ? L[2 * K1MAX + p2] : ~0ull, a3 = p3 < K1MAX ? L[3 * K1MAX + p3] : ~0ull;
+                uint64_t m01 = a0 < a1 ? a0 : a1, m23 = a2 < a3 ? a2 : a3;
+                const uint64_t mm = m01 < m23 ? m01 : m23;
+                if (mm == a0) ++p0;
+                else if (mm == a1) ++p1;
+                else if (mm == a2) ++p2;
+                else ++p3;
+                if (t < K) ids[t] = desc_key_index(mm);
+                if (t == K - 1) vk = desc_key_value(mm);
+                if (t == K) vk1 = desc_key_value(mm);
+            }
+            const int kk = min(K, nn);
+            // ids ascending (insertion sort of at most K1MAX - 1 values)
+            for (int a = 1; a < kk; ++a) {
+                const uint32_t x = ids[a];
+                int c = a - 1;
+                while (c >= 0 && ids[c] > x) {
+                    ids[c + 1] = ids[c];
+                    --c;
+                }
+                ids[c + 1] = x;
+            }
+            int *row = idx + (((size_t)b * D.Hkv + g) * D.T + ii) * K;
+            for (int t = 0; t < K; ++t) row[t] = t < kk ? (int)ids[t] : -1;
+            if (gap) gap[((size_t)b * D.Hkv + g) * D.T + ii] = (nn > K) ? vk - vk1 : INFINITY;
+        }
+    }
+    if (!ok && tid == 0) atomicOr(&g_select_tc_errors, 2u);
+}
+
+}  // namespace
+
+bool select_tc_supported(const Dims &D, int dtype) {
+    if (dtype != HILS_BF16 || D.d != 128 || D.G > 4 || D.topk > 32 || D.Nc < 1) return false;
+    const int n_max = window_left(D.q_pos0 + D.T - 1, D.W, D.S) / D.S;
+    return n_max >= 1 && n_max <= kRows;
+}
+
+unsigned int select_tc_error_flags(bool clear) {
+    unsigned int v = 0;
+    cudaMemcpyFromSymbol(&v, g_select_tc_errors, sizeof(v));
+    if (clear && v) {
+        const unsigned int zero = 0;
+        cudaMemcpyToSymbol(g_select_tc_errors, &zero, sizeof(zero));
+    }
+    return v;
+}
+
+cudaError_t launch_select_tc(const Dims &D, const void *q_hat, const void *k_sum, const float *b_sum, int *idx,
+                             float *gap, cudaStream_t stream) {
+    CUtensorMap qmap, kmap;
+    if (!make_tmap_bf16_2d(&qmap, q_hat, (uint64_t)D.B * D.Hq * D.T, 128, 128, 128) ||
+        !make_tmap_bf16_2d(&kmap, k_sum, (uint64_t)D.B * D.Hq * D.Nc, 128, 128, 128))
+        return cudaErrorInvalidValue;
+    dim3 grid((D.T + kRows - 1) / kRows, D.Hkv, D.B);
+    if (D.topk <= 16) {
+        const size_t smem = 1024 + 2 * (size_t)kStageBytes;  // lists: 128 * 4 * 17 * 8 = 68 KiB fit in the stages
+        cudaFuncSetAttribute(select_tc_kernel<17>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        select_tc_kernel<17><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap);
+    } else {
+        const size_t smem = 1024 + (size_t)kRows * 4 * 33 * 8;  // 132 KiB of lists > the two stages
+        cudaFuncSetAttribute(select_tc_kernel<33>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        select_tc_kernel<33><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace hils
