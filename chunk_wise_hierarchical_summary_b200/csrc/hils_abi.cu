@@ -18,7 +18,8 @@ cudaError_t launch_attn_fwd_simt(const Dims &D, int dtype, const void *q, const 
 bool attn_fwd_tc_supported(const Dims &D, int dtype);
 cudaError_t launch_attn_fwd_tc(const Dims &D, const void *q, const void *k, const void *v, const void *q_hat,
                                const void *k_sum, const float *b_sum, const int *idx, void *out, float *lse,
-                               cudaStream_t stream);
+                               void *ws, cudaStream_t stream);
+unsigned int attn_tc_error_flags(bool clear);
 size_t attn_fwd_tc_workspace(const Dims &D);
 hils_status check_device_errors();
 bool select_tc_supported(const Dims &D, int dtype);
@@ -97,6 +98,9 @@ hils_status check_device_errors() {
     if (select_tc_error_flags(true) != 0)
         return fail(HILS_ERR_TIMEOUT, "hils_check: a tensor-core selection tile's wait expired; that call's ids are "
                     "invalid");
+    if (attn_tc_error_flags(true) != 0)
+        return fail(HILS_ERR_TIMEOUT, "hils_check: a tensor-core attention tile's wait expired; that call's output "
+                    "is invalid");
     if (decode_error_flags(true) != 0)
         return fail(HILS_ERR_TIMEOUT, "hils_check: a decode tile's bulk copy did not complete within its wait "
                     "budget; that call's output is invalid");
@@ -201,7 +205,8 @@ hils_status hils_attn_fwd(const hils_params *p, const void *q, const void *k, co
     st = check_ws(fn, workspace, workspace_bytes, tc ? attn_fwd_tc_workspace(D) : 0);
     if (st != HILS_OK) return st;
     if (tc)
-        return cuda_status(launch_attn_fwd_tc(D, q, k, v, q_hat, k_sum, b_sum, idx, out, lse, (cudaStream_t)stream), fn);
+        return cuda_status(
+            launch_attn_fwd_tc(D, q, k, v, q_hat, k_sum, b_sum, idx, out, lse, workspace, (cudaStream_t)stream), fn);
     return cuda_status(
         launch_attn_fwd_simt(D, p->dtype, q, k, v, q_hat, k_sum, b_sum, idx, out, lse, (cudaStream_t)stream), fn);
 }

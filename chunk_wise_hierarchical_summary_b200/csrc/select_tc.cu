@@ -26,10 +26,11 @@ constexpr int kStageBytes = 65536;  // q^ tile (32 KiB) + k' tile (32 KiB)
 
 __device__ unsigned int g_select_tc_errors = 0;
 
-template <int K1MAX>
+template <int K1MAX, int GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
 select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, Dims D,
-                 const float *__restrict__ b_sum, int *__restrict__ idx, float *__restrict__ gap) {
+                 const float *__restrict__ b_sum, int *__restrict__ idx, float *__restrict__ gap,
+                 int *__restrict__ ws_idx, float *__restrict__ ws_shat) {
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t tma_bar[2], mma_bar[2], done_bar;
     __shared__ uint32_t s_tmem;
@@ -107,6 +108,65 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
     const int i = i0 + r;
     const int n_r = (i < D.T) ? window_left(D.q_pos0 + i, D.W, D.S) / D.S : 0;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+
+    if (GATHER) {
+        // Gather mode: row (query) r of head j reads its caller-given ids, keeps the valid distinct
+        // ones ascending and writes them with their retrieval scores s^ = tau D + b' to the workspace.
+        if (j < G) {  // warp-uniform: every lane executes the TMEM loads
+            const int hh = j, K = D.topk;
+            const bool valid = i < D.T;
+            int cl[32];
+            int ns = 0;
+            if (valid) {
+                const int *src = idx + (((size_t)b * D.Hkv + g) * D.T + i) * K;
+                for (int t = 0; t < K; ++t) {
+                    const int c = src[t];
+                    if (c < 0 || c >= n_r) continue;
+                    bool dup = false;
+                    for (int u = 0; u < ns; ++u) dup |= (cl[u] == c);
+                    if (dup) continue;
+                    int pos = ns;
+                    while (pos > 0 && cl[pos - 1] > c) {
+                        cl[pos] = cl[pos - 1];
+                        --pos;
+                    }
+                    cl[pos] = c;
+                    ++ns;
+                }
+            }
+            float *dst_s = ws_shat + (((size_t)b * D.Hq + g * G + hh) * D.T + i) * K;
+            int u = 0;
+#pragma unroll 1
+            for (int t = 0; t < 4; ++t) {
+                float v[32];
+                tmem_ld32(lane_base + hh * 128 + 32 * t, v);
+                tmem_wait_ld();
+                while (u < ns && cl[u] < 32 * t + 32) {
+                    const int e0 = cl[u] - 32 * t;
+                    float val = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) val = (e == e0) ? v[e] : val;
+                    dst_s[u] = fmaf(D.tau, val, bs[hh][cl[u]]);
+                    ++u;
+                }
+            }
+            if (valid) {
+                for (int t = ns; t < K; ++t) dst_s[t] = -INFINITY;
+                if (hh == 0) {
+                    int *dst_i = ws_idx + (((size_t)b * D.Hkv + g) * D.T + i) * K;
+                    for (int t = 0; t < K; ++t) dst_i[t] = t < ns ? cl[t] : -1;
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) {
+            tc_fence_after();
+            tmem_dealloc(tmem, ncols);
+        }
+        if (!ok && tid == 0) atomicOr(&g_select_tc_errors, 2u);
+        return;
+    }
 
     // Phase 1: per-head log-partition over the row's candidates.
     if (j < G) {
@@ -253,13 +313,29 @@ cudaError_t launch_select_tc(const Dims &D, const void *q_hat, const void *k_sum
     dim3 grid((D.T + kRows - 1) / kRows, D.Hkv, D.B);
     if (D.topk <= 16) {
         const size_t smem = 1024 + 2 * (size_t)kStageBytes;  // lists: 128 * 4 * 17 * 8 = 68 KiB fit in the stages
-        cudaFuncSetAttribute(select_tc_kernel<17>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        select_tc_kernel<17><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap);
+        cudaFuncSetAttribute(select_tc_kernel<17, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        select_tc_kernel<17, 0><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap, nullptr, nullptr);
     } else {
         const size_t smem = 1024 + (size_t)kRows * 4 * 33 * 8;  // 132 KiB of lists > the two stages
-        cudaFuncSetAttribute(select_tc_kernel<33>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        select_tc_kernel<33><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap);
+        cudaFuncSetAttribute(select_tc_kernel<33, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        select_tc_kernel<33, 0><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap, nullptr, nullptr);
     }
+    return cudaGetLastError();
+}
+
+// Canonical selection (valid distinct ids ascending, -1 padded) and the matching retrieval scores of
+// every (row, slot), for the tensor-core attention. Same GEMM as the selection; needs topk <= 32.
+cudaError_t launch_gather_shat_tc(const Dims &D, const void *q_hat, const void *k_sum, const float *b_sum,
+                                  const int *idx, int *ws_idx, float *ws_shat, cudaStream_t stream) {
+    CUtensorMap qmap, kmap;
+    if (!make_tmap_bf16_2d(&qmap, q_hat, (uint64_t)D.B * D.Hq * D.T, 128, 128, 128) ||
+        !make_tmap_bf16_2d(&kmap, k_sum, (uint64_t)D.B * D.Hq * D.Nc, 128, 128, 128))
+        return cudaErrorInvalidValue;
+    dim3 grid((D.T + kRows - 1) / kRows, D.Hkv, D.B);
+    const size_t smem = 1024 + 2 * (size_t)kStageBytes;
+    cudaFuncSetAttribute(select_tc_kernel<17, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    select_tc_kernel<17, 1><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, const_cast<int *>(idx), nullptr,
+                                                               ws_idx, ws_shat);
     return cudaGetLastError();
 }
 

@@ -116,7 +116,9 @@ HILS_API hils_status hils_select_topk(const hils_params *p, const void *q_hat, c
  *   lse = log Z^ = LSE({s_j}_window U {s^_c}_selected);
  *   out = sum_window exp(s_j - lse) v_j + sum_c exp(s^_c - lse) o_c.
  * The per-chunk outputs o_c never reach memory: each chunk's weights are scaled by
- * exp(s^_c - L_c) before its value product. fp32 accumulation. Workspace: none.
+ * exp(s^_c - L_c) before its value product. fp32 accumulation.
+ * Workspace: hils_workspace_size(p, HILS_OP_ATTN_FWD) bytes (non-zero on the tensor-core path:
+ * bf16, d 128, S 64, G <= 4, topk <= 32, at most 128 candidate chunks per row).
  */
 HILS_API hils_status hils_attn_fwd(const hils_params *p, const void *q, const void *k, const void *v, const void *q_hat,
                           const void *k_sum, const float *b_sum, const int32_t *idx, void *out, float *lse,
