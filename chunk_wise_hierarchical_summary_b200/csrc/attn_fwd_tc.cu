@@ -35,21 +35,49 @@ bool select_tc_supported(const Dims &D, int dtype);
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kStages = 3;
+constexpr int kStages = 2;           // K ring and V ring, each kStages deep
 constexpr int kListCap = 1024;
-constexpr int kBitmapWords = 2048;  // chunks per sequence <= 65536
+constexpr int kBitmapWords = 256;    // chunks per sequence <= 8192
 constexpr uint32_t kQBytes = 32768;
-constexpr uint32_t kKVBytes = 32768;  // K tile 16 KiB + V tile 16 KiB
-constexpr uint32_t kPBytes = 16384;
-constexpr float kRescaleSlack = 8.f;
+constexpr uint32_t kTileBytes = 16384;  // one K or V tile: 64 tokens x 128 d bf16
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleSlack2 = 11.5f;  // log2 units (about 8 in natural units)
 
 __device__ unsigned int g_attn_tc_errors = 0;
 
 struct Bars {
-    uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], s_free[2], p_full, pv_done;
+    // p_full is per S/P buffer: a row warp may run one tile ahead (its next S is ready before every warp
+    // has written this tile's P), so one shared barrier would let an early arrival complete a phase.
+    // o_final completes once, after the last value product: the row warps' epilogue cannot wait on a
+    // pv_done parity, because a warp that skipped per-tile waits may see pv_done two phases behind.
+    uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages], s_full[2], p_full[2],
+        pv_done, o_final;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+// D += A(TMEM) x B(smem descriptor): the P V product with P read from TMEM (K-major by construction).
+__device__ __forceinline__ void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                const __grid_constant__ CUtensorMap vmap, Dims D, const int *__restrict__ ws_idx,
                const float *__restrict__ ws_shat, __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
@@ -65,27 +93,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     const int S = D.S, K = D.topk;
     unsigned char *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     unsigned char *Qs = base;
-    unsigned char *KV = base + kQBytes;
-    unsigned char *Ps = KV + kStages * kKVBytes;
+    unsigned char *Ks = base + kQBytes;                    // kStages K tiles
+    unsigned char *Vs = Ks + kStages * kTileBytes;         // kStages V tiles
     const int nchunks = (D.L + S - 1) / S;
     const int nwords = (nchunks + 31) / 32;
+    const float scale2 = D.tau * kLog2e;
 
     if (warp == 1) {
-        tmem_alloc(&s_tmem, 256);
+        tmem_alloc(&s_tmem, 256);  // S/P buffers: columns [0,64) and [64,128); O: [128,256)
         tmem_relinquish();
     }
     if (tid == 0) {
         mbar_init(&bar.q_full, 1);
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&bar.kv_full[s], 1);
-            mbar_init(&bar.kv_empty[s], 1);
+            mbar_init(&bar.k_full[s], 1);
+            mbar_init(&bar.k_empty[s], 1);
+            mbar_init(&bar.v_full[s], 1);
+            mbar_init(&bar.v_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bar.s_full[s], 1);
-            mbar_init(&bar.s_free[s], 128);
+            mbar_init(&bar.p_full[s], 128);
         }
-        mbar_init(&bar.p_full, 128);
         mbar_init(&bar.pv_done, 1);
+        mbar_init(&bar.o_final, 1);
         fence_mbar_init();
     }
     for (int w = tid; w < nwords; w += blockDim.x) bitmap[w] = 0;
@@ -106,13 +137,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     const int *row_idx = ws_idx + (((size_t)b * D.Hkv + g) * D.T + (valid ? i : 0)) * K;
     const float *row_sh = ws_shat + (((size_t)b * D.Hq + g * G + hh) * D.T + (valid ? i : 0)) * K;
     int ns = 0;
-    float m_run = -INFINITY;
+    float m2 = -INFINITY;  // running max, log2 units
     if (valid) {
         for (int t = 0; t < K; ++t) {
             const int c = row_idx[t];
             if (c < 0) break;
             ++ns;
-            m_run = fmaxf(m_run, row_sh[t]);
+            m2 = fmaxf(m2, row_sh[t] * kLog2e);
             atomicOr(&bitmap[c >> 5], 1u << (c & 31));
         }
     }
@@ -140,25 +171,36 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
+        // K of tile n and V of tile n-1 per step, so K loads run ahead of the value products.
         if (lane == 0) {
             const int head0 = b * D.Hq + g * G;
             mbar_arrive_expect_tx(&bar.q_full, kQBytes);
             tma_load_3d(Qs, &qmap, 0, head0, i0, &bar.q_full);
             tma_load_3d(Qs + 16384, &qmap, 64, head0, i0, &bar.q_full);
             const int kvrow0 = (b * D.Hkv + g) * D.L;
-            for (int n = 0; n < ntiles && ok; ++n) {
+            auto load_k = [&](int n) {
                 const int st = n % kStages;
-                if (n >= kStages && !mbar_wait_bounded(&bar.kv_empty[st], ((n / kStages) - 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                unsigned char *Kt = KV + st * kKVBytes, *Vt = Kt + 16384;
+                if (n >= kStages && !mbar_wait_bounded(&bar.k_empty[st], ((n / kStages) - 1) & 1)) return false;
+                unsigned char *Kt = Ks + st * kTileBytes;
                 const int y = kvrow0 + list[n] * S;
-                mbar_arrive_expect_tx(&bar.kv_full[st], kKVBytes);
-                tma_load_2d(Kt, &kmap, 0, y, &bar.kv_full[st]);
-                tma_load_2d(Kt + 8192, &kmap, 64, y, &bar.kv_full[st]);
-                tma_load_2d(Vt, &vmap, 0, y, &bar.kv_full[st]);
-                tma_load_2d(Vt + 8192, &vmap, 64, y, &bar.kv_full[st]);
+                mbar_arrive_expect_tx(&bar.k_full[st], kTileBytes);
+                tma_load_2d(Kt, &kmap, 0, y, &bar.k_full[st]);
+                tma_load_2d(Kt + 8192, &kmap, 64, y, &bar.k_full[st]);
+                return true;
+            };
+            auto load_v = [&](int n) {
+                const int st = n % kStages;
+                if (n >= kStages && !mbar_wait_bounded(&bar.v_empty[st], ((n / kStages) - 1) & 1)) return false;
+                unsigned char *Vt = Vs + st * kTileBytes;
+                const int y = kvrow0 + list[n] * S;
+                mbar_arrive_expect_tx(&bar.v_full[st], kTileBytes);
+                tma_load_2d(Vt, &vmap, 0, y, &bar.v_full[st]);
+                tma_load_2d(Vt + 8192, &vmap, 64, y, &bar.v_full[st]);
+                return true;
+            };
+            for (int n = 0; n <= ntiles && ok; ++n) {
+                if (n < ntiles && !load_k(n)) ok = false;
+                if (ok && n >= 1 && !load_v(n - 1)) ok = false;
             }
         }
         __syncwarp();
@@ -167,24 +209,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         if (lane == 0) {
             const uint32_t idesc_qk = idesc_bf16_f32(128, 64, 0, 0);
             const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
-            const uint32_t qa = smem_u32(Qs), pa = smem_u32(Ps);
+            const uint32_t qa = smem_u32(Qs);
             ok = mbar_wait_bounded(&bar.q_full, 0);
             auto issue_pv = [&](int n) {
                 const int st = n % kStages;
-                const uint32_t va = smem_u32(KV + st * kKVBytes + 16384);
+                if (!mbar_wait_bounded(&bar.v_full[st], (n / kStages) & 1)) return false;
+                tc_fence_after();
+                const uint32_t va = smem_u32(Vs + st * kTileBytes);
+                const uint32_t pa = tmem + (n & 1) * 64;  // P(n) aliases S(n): 32 columns of bf16 pairs
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    umma_bf16(tmem + 128, sdesc_sw128(pa + ks * 32, 16, 1024), sdesc_sw128(va + ks * 2048, 8192, 1024),
-                              idesc_pv, (n > 0 || ks > 0) ? 1u : 0u);
+                    umma_bf16_tmem_a(tmem + 128, pa + ks * 8, sdesc_sw128(va + ks * 2048, 8192, 1024), idesc_pv,
+                                     (n > 0 || ks > 0) ? 1u : 0u);
                 umma_commit(&bar.pv_done);
-                umma_commit(&bar.kv_empty[st]);
+                umma_commit(&bar.v_empty[st]);
+                return true;
             };
             for (int n = 0; n < ntiles && ok; ++n) {
                 const int st = n % kStages, sb = n & 1;
-                if (!mbar_wait_bounded(&bar.kv_full[st], (n / kStages) & 1)) { ok = false; break; }
-                if (n >= 2 && !mbar_wait_bounded(&bar.s_free[sb], ((n >> 1) - 1) & 1)) { ok = false; break; }
+                if (!mbar_wait_bounded(&bar.k_full[st], (n / kStages) & 1)) { ok = false; break; }
+                // S/P buffer sb held P(n-2): reuse it only after PV(n-2) has completed
+                if (n >= 2 && !mbar_wait_bounded(&bar.pv_done, (n - 2) & 1)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t ka = smem_u32(KV + st * kKVBytes);
+                const uint32_t ka = smem_u32(Ks + st * kTileBytes);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
@@ -193,20 +240,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                               idesc_qk, ks > 0 ? 1u : 0u);
                 }
                 umma_commit(&bar.s_full[sb]);
+                umma_commit(&bar.k_empty[st]);
                 if (n >= 1) {
-                    if (!mbar_wait_bounded(&bar.p_full, (n - 1) & 1)) { ok = false; break; }
+                    if (!mbar_wait_bounded(&bar.p_full[(n - 1) & 1], ((n - 1) >> 1) & 1)) { ok = false; break; }
                     tc_fence_after();
-                    issue_pv(n - 1);
+                    if (!issue_pv(n - 1)) { ok = false; break; }
                 }
             }
             if (ok && ntiles > 0) {
-                if (mbar_wait_bounded(&bar.p_full, (ntiles - 1) & 1)) {
+                if (mbar_wait_bounded(&bar.p_full[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1)) {
                     tc_fence_after();
-                    issue_pv(ntiles - 1);
+                    if (!issue_pv(ntiles - 1)) ok = false;
                 } else {
                     ok = false;
                 }
             }
+            umma_commit(&bar.o_final);  // arrives once every MMA above has completed (also on error paths)
         }
         __syncwarp();
     } else {
@@ -214,17 +263,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16);
         float l_run = 0.f;
         int u = ns - 1;  // cursor into the row's ascending chunk list (tiles arrive descending)
+        int cur_c = (valid && u >= 0) ? row_idx[u] : -1;
+        float cur_sh2 = (valid && u >= 0) ? row_sh[u] * kLog2e : 0.f;
         for (int n = 0; n < ntiles; ++n) {
             const int sb = n & 1;
             const int c = list[n];
-            float v[64];
-            // a failed wait ends the row loop of the whole warp (the wait result is warp-uniform in practice,
-            // and the ballot makes it so)
             if (__any_sync(0xffffffffu, !mbar_wait_bounded(&bar.s_full[sb], (n >> 1) & 1))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
+            float v[64];
             {
                 float a[32];
                 tmem_ld32(lane_base + sb * 64, a);
@@ -235,96 +284,76 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                 for (int e = 0; e < 32; ++e) v[32 + e] = a[e];
                 tmem_wait_ld();
             }
-            tc_fence_before();
-            mbar_arrive(&bar.s_free[sb]);
-            // role of this row for chunk c
-            while (u >= 0 && row_idx[u] > c) --u;
-            const bool sel = valid && u >= 0 && row_idx[u] == c;
+            while (cur_c > c) {
+                --u;
+                cur_c = u >= 0 ? row_idx[u] : -1;
+                cur_sh2 = u >= 0 ? row_sh[u] * kLog2e : 0.f;
+            }
+            const bool sel = valid && cur_c == c;
             const int j0 = c * S;
             const bool win = valid && !sel && j0 <= pos && j0 + S - 1 >= lpos;
-            float tmax = -INFINITY;
-            if (sel) {
-                float mx = -INFINITY;
+            // pass 1: mask and raw max
+            float mraw = -INFINITY;
 #pragma unroll
-                for (int e = 0; e < 64; ++e) {
-                    v[e] *= D.tau;
-                    mx = fmaxf(mx, v[e]);
-                }
-                float z = 0.f;
-#pragma unroll
-                for (int e = 0; e < 64; ++e) z += __expf(v[e] - mx);
-                const float off = row_sh[u] - (mx + logf(z));
-#pragma unroll
-                for (int e = 0; e < 64; ++e) v[e] += off;
-                tmax = mx + off;
-            } else if (win) {
-#pragma unroll
-                for (int e = 0; e < 64; ++e) {
-                    const int jj = j0 + e;
-                    v[e] = (jj >= lpos && jj <= pos) ? v[e] * D.tau : -INFINITY;
-                    tmax = fmaxf(tmax, v[e]);
-                }
+            for (int e = 0; e < 64; ++e) {
+                const int jj = j0 + e;
+                const bool keep = sel || (win && jj >= lpos && jj <= pos);
+                v[e] = keep ? v[e] : -INFINITY;
+                mraw = fmaxf(mraw, v[e]);
             }
+            const float tmax = mraw * scale2;  // tau > 0: the max commutes with the scale
             float factor = 1.f;
-            if (tmax > m_run + kRescaleSlack || (m_run == -INFINITY && tmax > -INFINITY)) {
-                const float m_new = fmaxf(tmax, m_run);
-                factor = (m_run == -INFINITY) ? 0.f : __expf(m_run - m_new);
+            if (win && (tmax > m2 + kRescaleSlack2 || (m2 == -INFINITY && tmax > -INFINITY))) {
+                const float m_new = fmaxf(tmax, m2);
+                factor = (m2 == -INFINITY) ? 0.f : exp2f(m2 - m_new);
                 l_run *= factor;
-                m_run = m_new;
+                m2 = m_new;
             }
-            // P in bf16; row sum in fp32
+            // pass 2: e_j = 2^(t_j - base); selected rows use the chunk max as base, others the running max
+            const float basev = sel ? tmax : (m2 == -INFINITY ? 0.f : m2);
+            float z = 0.f;
+#pragma unroll
+            for (int e = 0; e < 64; ++e) {
+                v[e] = exp2f(fmaf(v[e], scale2, -basev));
+                z += v[e];
+            }
+            // selected chunk: total mass 2^(s^2 - m2), split by the intra-chunk softmax e_j / z
+            const float f = sel ? exp2f(cur_sh2 - m2) / z : 1.f;
+            l_run += z * f;
             uint32_t pk[32];
-            float psum = 0.f;
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-                const float p0 = (sel || win) ? __expf(v[2 * e] - m_run) : 0.f;
-                const float p1 = (sel || win) ? __expf(v[2 * e + 1] - m_run) : 0.f;
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * e] * f, v[2 * e + 1] * f);
                 pk[e] = *reinterpret_cast<const uint32_t *>(&h2);
-                psum += p0 + p1;
             }
-            l_run += psum;
-            // P buffer and O are free once PV(n-1) has completed
-            if (n >= 1) {
+            // O rescale (rare; warp-collective TMEM access) once PV(n-1) has completed
+            const unsigned need = __ballot_sync(0xffffffffu, factor != 1.f && n >= 1);
+            if (need) {
                 if (__any_sync(0xffffffffu, !mbar_wait_bounded(&bar.pv_done, (n - 1) & 1))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-            }
-            {
-                // TMEM loads/stores are warp-collective: the whole warp rescales if any of its rows needs it
-                // (rows that do not need it multiply by 1).
-                const unsigned need = __ballot_sync(0xffffffffu, factor != 1.f && n >= 1);
-                if (need) {
 #pragma unroll 1
-                    for (int t = 0; t < 4; ++t) {
-                        float o[32];
-                        tmem_ld32(lane_base + 128 + 32 * t, o);
-                        tmem_wait_ld();
+                for (int t = 0; t < 4; ++t) {
+                    float o[32];
+                    tmem_ld32(lane_base + 128 + 32 * t, o);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] *= factor;
-                        tmem_st32(lane_base + 128 + 32 * t, o);
-                    }
-                    tmem_wait_st();
+                    for (int e = 0; e < 32; ++e) o[e] *= factor;
+                    tmem_st32(lane_base + 128 + 32 * t, o);
                 }
             }
-            // P row r, 128 bytes, 16-byte chunk k stored at chunk k ^ (r % 8)
-            unsigned char *prow = Ps + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                uint4 w4 = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
-                *reinterpret_cast<uint4 *>(prow + ((k ^ (r & 7)) << 4)) = w4;
-            }
-            fence_async_smem();
+            // P(n) over S(n) in TMEM (S(n) is read; PV(n-2), the last reader of these columns, completed
+            // before QK(n) was issued)
+            tmem_st32u(lane_base + sb * 64, pk);
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bar.p_full);
+            mbar_arrive(&bar.p_full[sb]);
         }
         // epilogue
-        if (ok && ntiles > 0) {
-            if (__any_sync(0xffffffffu, !mbar_wait_bounded(&bar.pv_done, (ntiles - 1) & 1))) ok = false;
-            tc_fence_after();
-        }
+        if (__any_sync(0xffffffffu, !mbar_wait_bounded(&bar.o_final, 0))) ok = false;
+        tc_fence_after();
         const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
         __nv_bfloat16 *orow = out + (((size_t)b * D.Hq + g * G + hh) * D.T + (valid ? i : 0)) * 128;
 #pragma unroll 1
@@ -345,7 +374,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                 }
             }
         }
-        if (valid) lse[((size_t)b * D.Hq + g * G + hh) * D.T + i] = m_run + logf(l_run);
+        if (valid) lse[((size_t)b * D.Hq + g * G + hh) * D.T + i] = (m2 + log2f(l_run)) * (1.f / kLog2e);
     }
     if (!ok) atomicOr(&g_attn_tc_errors, 1u);
     tc_fence_before();
@@ -400,7 +429,7 @@ cudaError_t launch_attn_fwd_tc(const Dims &D, const void *q, const void *k, cons
         !make_tmap_bf16_2d(&kmap, k, (uint64_t)D.B * D.Hkv * D.L, 128, 128, 64) ||
         !make_tmap_bf16_2d(&vmap, v, (uint64_t)D.B * D.Hkv * D.L, 128, 128, 64))
         return cudaErrorInvalidValue;
-    const size_t smem = 1024 + kQBytes + kStages * kKVBytes + kPBytes;
+    const size_t smem = 1024 + kQBytes + 2 * kStages * kTileBytes;
     cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     dim3 grid((D.T + QT - 1) / QT, D.Hkv, D.B);
     attn_tc_kernel<<<grid, kThreads, smem, stream>>>(qmap, kmap, vmap, D, ws_idx, ws_shat, (__nv_bfloat16 *)out, lse);
