@@ -65,6 +65,13 @@ __device__ __forceinline__ void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tme
         : "memory");
 }
 
+// 2^x on the special-function unit (PTX ex2.approx.ftz); 2^-inf = 0.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -261,70 +268,105 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     } else {
         // ---------------------------------------------------------------- one row per thread
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16);
+        const float2 sc2 = make_float2(scale2, scale2);
         float l_run = 0.f;
-        int u = ns - 1;  // cursor into the row's ascending chunk list (tiles arrive descending)
+        // Cursor into the row's ascending chunk list, walked from the top because tiles arrive in
+        // descending order. Every selected chunk is in the tile list, so the current entry is matched by
+        // equality; the entry after it is loaded one match ahead, off the critical path.
+        int u = ns - 1;
         int cur_c = (valid && u >= 0) ? row_idx[u] : -1;
         float cur_sh2 = (valid && u >= 0) ? row_sh[u] * kLog2e : 0.f;
+        int nxt_c = (valid && u >= 1) ? row_idx[u - 1] : -1;
+        float nxt_sh2 = (valid && u >= 1) ? row_sh[u - 1] * kLog2e : 0.f;
         for (int n = 0; n < ntiles; ++n) {
             const int sb = n & 1;
             const int c = list[n];
+            const int j0 = c * S;
+            const bool sel = valid && cur_c == c;
+            int lo = 0, hi = S - 1;
+            if (valid && !sel) {
+                lo = max(lpos - j0, 0);
+                hi = min(pos - j0, S - 1);
+            }
+            const bool win = valid && !sel && lo <= hi;
+            const float sh2 = cur_sh2;
+            if (sel) {
+                cur_c = nxt_c;
+                cur_sh2 = nxt_sh2;
+                --u;
+                nxt_c = u >= 1 ? row_idx[u - 1] : -1;
+                nxt_sh2 = u >= 1 ? row_sh[u - 1] * kLog2e : 0.f;
+            }
             if (__any_sync(0xffffffffu, !mbar_wait_bounded(&bar.s_full[sb], (n >> 1) & 1))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            float v[64];
-            {
-                float a[32];
-                tmem_ld32(lane_base + sb * 64, a);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = a[e];
-                tmem_ld32(lane_base + sb * 64 + 32, a);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) v[32 + e] = a[e];
-                tmem_wait_ld();
-            }
-            while (cur_c > c) {
-                --u;
-                cur_c = u >= 0 ? row_idx[u] : -1;
-                cur_sh2 = u >= 0 ? row_sh[u] * kLog2e : 0.f;
-            }
-            const bool sel = valid && cur_c == c;
-            const int j0 = c * S;
-            const bool win = valid && !sel && j0 <= pos && j0 + S - 1 >= lpos;
-            // pass 1: mask and raw max
-            float mraw = -INFINITY;
-#pragma unroll
-            for (int e = 0; e < 64; ++e) {
-                const int jj = j0 + e;
-                const bool keep = sel || (win && jj >= lpos && jj <= pos);
-                v[e] = keep ? v[e] : -INFINITY;
-                mraw = fmaxf(mraw, v[e]);
-            }
-            const float tmax = mraw * scale2;  // tau > 0: the max commutes with the scale
-            float factor = 1.f;
-            if (win && (tmax > m2 + kRescaleSlack2 || (m2 == -INFINITY && tmax > -INFINITY))) {
-                const float m_new = fmaxf(tmax, m2);
-                factor = (m2 == -INFINITY) ? 0.f : exp2f(m2 - m_new);
-                l_run *= factor;
-                m2 = m_new;
-            }
-            // pass 2: e_j = 2^(t_j - base); selected rows use the chunk max as base, others the running max
-            const float basev = sel ? tmax : (m2 == -INFINITY ? 0.f : m2);
-            float z = 0.f;
-#pragma unroll
-            for (int e = 0; e < 64; ++e) {
-                v[e] = exp2f(fmaf(v[e], scale2, -basev));
-                z += v[e];
-            }
-            // selected chunk: total mass 2^(s^2 - m2), split by the intra-chunk softmax e_j / z
-            const float f = sel ? exp2f(cur_sh2 - m2) / z : 1.f;
-            l_run += z * f;
             uint32_t pk[32];
+            float factor = 1.f;
+            if (__any_sync(0xffffffffu, sel || win)) {
+                float v[64];
+                {
+                    float a[32];
+                    tmem_ld32(lane_base + sb * 64, a);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * e] * f, v[2 * e + 1] * f);
-                pk[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                    for (int e = 0; e < 32; ++e) v[e] = a[e];
+                    tmem_ld32(lane_base + sb * 64 + 32, a);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[32 + e] = a[e];
+                    tmem_wait_ld();
+                }
+                // only a window row whose window starts or ends inside this tile needs a mask
+                if (__any_sync(0xffffffffu, win && (lo > 0 || hi < S - 1))) {
+                    const int mlo = win ? lo : 0, mhi = win ? hi : S - 1;
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) v[e] = (e >= mlo && e <= mhi) ? v[e] : -INFINITY;
+                }
+                float mx[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) mx[e] = v[e];
+#pragma unroll
+                for (int e = 8; e < 64; ++e) mx[e & 7] = fmaxf(mx[e & 7], v[e]);
+                const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                const float tmax = mraw * scale2;  // tau > 0: the max commutes with the scale
+                if (win && tmax > m2 + kRescaleSlack2) {
+                    // a row with no mass yet (m2 = -inf) has O = 0 and l = 0: no rescale needed
+                    if (m2 != -INFINITY) factor = ex2_approx(m2 - tmax);
+                    l_run *= factor;
+                    m2 = tmax;
+                }
+                // e_j = 2^(t_j - base): window rows use the running max, all others their tile max
+                const float basev = win ? m2 : tmax;
+                const float2 nb2 = make_float2(-basev, -basev);
+                float2 zacc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                  make_float2(0.f, 0.f)};
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    float2 t = __ffma2_rn(make_float2(v[2 * e], v[2 * e + 1]), sc2, nb2);
+                    t.x = ex2_approx(t.x);
+                    t.y = ex2_approx(t.y);
+                    v[2 * e] = t.x;
+                    v[2 * e + 1] = t.y;
+                    zacc[e & 3] = __fadd2_rn(zacc[e & 3], t);
+                }
+                const float2 zz = __fadd2_rn(__fadd2_rn(zacc[0], zacc[1]), __fadd2_rn(zacc[2], zacc[3]));
+                const float z = zz.x + zz.y;
+                // selected chunk: total mass 2^(s^2 - m2), split by the intra-chunk softmax e_j / z;
+                // a row that neither selects nor windows this tile contributes P = 0
+                const float mass = sel ? ex2_approx(sh2 - m2) : 0.f;
+                const float f = sel ? mass / z : (win ? 1.f : 0.f);
+                l_run += win ? z : mass;
+                const float2 f2 = make_float2(f, f);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const float2 pr = __fmul2_rn(make_float2(v[2 * e], v[2 * e + 1]), f2);
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(pr.x, pr.y);
+                    pk[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) pk[e] = 0u;
             }
             // O rescale (rare; warp-collective TMEM access) once PV(n-1) has completed
             const unsigned need = __ballot_sync(0xffffffffu, factor != 1.f && n >= 1);
