@@ -137,6 +137,19 @@ class Dist:
             self.pg.destroy_process_group()
 
 
+def weak_scaling_value(dist: Dist, ms_local: float, units_per_rank: float):
+    """Whole-job throughput under weak scaling: every rank processes `units_per_rank` independent units
+    (its own sequences; no data-path collective), and the job takes as long as its slowest rank.
+    Returns (max-over-ranks milliseconds, units per second over all ranks)."""
+    ms = dist.max(ms_local)
+    return ms, dist.world * units_per_rank / (ms / 1e3)
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Seed of a rank's synthetic inputs: ranks draw distinct sequences of the same shapes."""
+    return base + rank
+
+
 def physical_gpu_index(local_rank: int) -> int:
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     if vis:
@@ -226,7 +239,7 @@ def decode_bytes(w: W.Workload):
 
 def bench_prefill(args, dist, dev, H, peaks):
     w = W.PREFILL_BF16
-    x = W.prefill_inputs(w, seed=1000 + dist.rank, device=dev)
+    x = W.prefill_inputs(w, seed=rank_seed(1000, dist.rank), device=dev)
     k_sum = torch.empty((w.B, w.Hq, w.Nc, w.d), dtype=torch.bfloat16, device=dev)
     b_sum = torch.empty((w.B, w.Hq, w.Nc), dtype=torch.float32, device=dev)
     idx = torch.empty((w.B, w.Hkv, w.T, w.topk), dtype=torch.int32, device=dev)
@@ -288,13 +301,13 @@ def bench_prefill_e2e(args, dist, dev, H, res):
         mark()
 
     _, total_ms, _ = timed_steps(steps, step, 2, None, dist)
-    ms = dist.max(total_ms / steps)
-    return {"value": dist.world * w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+    ms, value = weak_scaling_value(dist, total_ms / steps, w.B * w.T)
+    return {"value": value, "unit": "tokens/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
 def bench_decode(args, dist, dev, H, peaks, w: W.Workload, steps: int):
-    x = W.decode_inputs(w, seed=2000 + dist.rank, device=dev)
+    x = W.decode_inputs(w, seed=rank_seed(2000, dist.rank), device=dev)
     k_sum, b_sum = H.chunk_summary(x["k_cache"], x["q_land"], w.S)
     out = torch.empty_like(x["q"])
     lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
@@ -328,7 +341,7 @@ def bench_decode(args, dist, dev, H, peaks, w: W.Workload, steps: int):
     needles_found = 0
     for b in range(w.B):
         needles_found += len(set(x["needle_chunks"][b].tolist()) & set(idx[b, 0].tolist()))
-    ms_step = total_ms / steps
+    ms_step = dist.max(total_ms / steps)  # per-sequence-batch latency: the slowest rank's
     nbytes = decode_bytes(w)
     gbs = nbytes["total"] / (ms_step / 1e3) / 1e9
     del graph
@@ -343,7 +356,7 @@ def bench_decode(args, dist, dev, H, peaks, w: W.Workload, steps: int):
 
 def bench_train(args, dist, dev, H, peaks):
     w = W.TRAIN_BF16
-    x = W.prefill_inputs(w, seed=3000 + dist.rank, device=dev, with_dout=True)
+    x = W.prefill_inputs(w, seed=rank_seed(3000, dist.rank), device=dev, with_dout=True)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def step(mark):
@@ -359,8 +372,8 @@ def bench_train(args, dist, dev, H, peaks):
     work = prefill_work(w)
     fwd_flops = work["attn_flops"] + work["route_flops"] + work["summary_flops"]
     bwd_flops = work["attn_flops"] * 14 // 4 + 2 * work["summary_flops"]
-    ms = total_ms / steps
-    return {"workload": w.name, "tokens_per_s": w.B * w.T / (ms / 1e3), "ms_per_step": ms,
+    ms, tps = weak_scaling_value(dist, total_ms / steps, w.B * w.T)
+    return {"workload": w.name, "tokens_per_s": tps, "ms_per_step": ms,
             "fwd_ms": stage_ms[0] / steps, "bwd_ms": stage_ms[1] / steps,
             "roofline": {"bound": "tensor", "kernel": "hils_attn_bwd",
                          "achieved": bwd_flops / (stage_ms[1] / steps / 1e3) / 1e12,
@@ -479,8 +492,7 @@ def main():
         peaks, peak_src = load_peaks()
         pre = bench_prefill(args, dist, dev, H, peaks)
         w = pre["workload"]
-        ms = dist.max(pre["ms_per_step"])
-        value = dist.world * w.B * w.T / (ms / 1e3)
+        ms, value = weak_scaling_value(dist, pre["ms_per_step"], w.B * w.T)
         e2e = bench_prefill_e2e(args, dist, dev, H, pre)
         decode = bench_decode(args, dist, dev, H, peaks, W.DECODE_BF16, 256)
         extra = {}
