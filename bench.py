@@ -309,6 +309,15 @@ def bench_prefill_e2e(args, dist, dev, H, res):
 def bench_decode(args, dist, dev, H, peaks, w: W.Workload, steps: int):
     x = W.decode_inputs(w, seed=rank_seed(2000, dist.rank), device=dev)
     k_sum, b_sum = H.chunk_summary(x["k_cache"], x["q_land"], w.S)
+    # the cache's summaries (stage (a)), timed once more on their own: K + landmark queries in, k' + b' out
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    H.chunk_summary(x["k_cache"], x["q_land"], w.S, k_sum=k_sum, b_sum=b_sum)
+    e1.record()
+    torch.cuda.synchronize()
+    summ_ms = e0.elapsed_time(e1)
+    el = 2 if w.dtype == "bf16" else 4
+    summ_bytes = (w.B * w.Hkv * w.Nc * w.S * w.d * el + 2 * w.B * w.Hq * w.Nc * w.d * el + 4 * w.B * w.Hq * w.Nc)
     out = torch.empty_like(x["q"])
     lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
     idx = torch.empty((w.B, w.Hkv, w.topk), dtype=torch.int32, device=dev)
@@ -345,7 +354,11 @@ def bench_decode(args, dist, dev, H, peaks, w: W.Workload, steps: int):
     nbytes = decode_bytes(w)
     gbs = nbytes["total"] / (ms_step / 1e3) / 1e9
     del graph
+    summ = {"ms": summ_ms, "bytes": summ_bytes, "achieved_gbs": summ_bytes / (summ_ms / 1e3) / 1e9,
+            "peak_gbs": peaks["hbm_gbs"], "frac": summ_bytes / (summ_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "note": "hils_chunk_summary over the whole cache: K and landmark queries read, k' and b' written"}
     return {"workload": w.name, "us_per_token": ms_step * 1e3, "us_per_step_per_seq": ms_step * 1e3 / w.B,
+            "summaries": summ,
             "steps": steps, "bytes_per_step": nbytes,
             "roofline": {"bound": "hbm", "kernel": "hils_decode (whole step: score, select, attend, combine)",
                          "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
@@ -468,6 +481,47 @@ def run_reference(args, dist):
     print(json.dumps(line))
 
 
+# ----------------------------------------------------------------------------- profiling cases
+
+def profile_case(args):
+    """`--profile STAGE`: `args.steps` untimed launches of one stage on its workload, for ncu captures of
+    one kernel (select it with ncu's -k / -s / -c). Prints no bench line. The summary case runs on a
+    128K-token cache (B1; 256 MiB of keys, above L2), the decode case on the 512K decode workload."""
+    import chunk_wise_hierarchical_summary_b200.hils as H
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    st = args.profile
+    if st in ("summary", "decode"):
+        w = W.DECODE_BF16 if st == "decode" else W.decode_sweep(131072)
+        x = W.decode_inputs(w, seed=2000, device=dev)
+        k_sum, b_sum = H.chunk_summary(x["k_cache"], x["q_land"], w.S)
+        if st == "summary":
+            fn = lambda: H.chunk_summary(x["k_cache"], x["q_land"], w.S, k_sum=k_sum, b_sum=b_sum)
+        else:
+            fn = lambda: H.decode(x["q"], x["q_hat"], x["k_cache"], x["v_cache"], k_sum, b_sum, S=w.S, topk=w.topk,
+                                  window=w.W)
+    else:
+        w = W.TRAIN_BF16 if st == "bwd" else W.PREFILL_BF16
+        x = W.prefill_inputs(w, seed=1000, device=dev, with_dout=(st == "bwd"))
+        out, lse, idx, k_sum, b_sum = H.prefill(x["q"], x["k"], x["v"], x["q_hat"], x["q_land"], S=w.S, topk=w.topk,
+                                                window=w.W)
+        if st == "select":
+            fn = lambda: H.select_topk(x["q_hat"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S, topk=w.topk, window=w.W,
+                                       idx=idx)
+        elif st == "attn":
+            fn = lambda: H.attn_fwd(x["q"], x["k"], x["v"], x["q_hat"], k_sum, b_sum, idx, S=w.S, window=w.W,
+                                    out=out, lse=lse)
+        else:
+            fn = lambda: H.attn_bwd(x["q"], x["k"], x["v"], x["q_hat"], x["q_land"], k_sum, b_sum, idx, out, lse,
+                                    x["dout"], S=w.S, window=w.W)
+    for _ in range(args.steps):
+        fn()
+    torch.cuda.synchronize()
+    H.check()
+    print(f"profile case {st} on {w.name}: {args.steps} launches done")
+
+
 # ----------------------------------------------------------------------------- main
 
 def main():
@@ -477,7 +531,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="hils", choices=("hils", "reference"))
     ap.add_argument("--quick", action="store_true", help="headline only (no decode sweep / training blocks)")
+    ap.add_argument("--profile", choices=("summary", "select", "attn", "decode", "bwd"),
+                    help="run --steps untimed launches of one stage for an ncu capture; no bench line")
     args = ap.parse_args()
+    if args.profile:
+        profile_case(args)
+        return
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     dist = Dist(args.gpus)

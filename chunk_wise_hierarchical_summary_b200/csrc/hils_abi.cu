@@ -26,6 +26,7 @@ bool select_tc_supported(const Dims &D, int dtype);
 cudaError_t launch_select_tc(const Dims &D, const void *q_hat, const void *k_sum, const float *b_sum, int *idx,
                              float *gap, cudaStream_t stream);
 unsigned int select_tc_error_flags(bool clear);
+unsigned int summary_error_flags(bool clear);
 
 namespace {
 
@@ -95,6 +96,9 @@ hils_status check_ws(const char *fn, void *ws, size_t have, size_t need) {
 void record_error(const char *msg) { g_last_error = msg; }
 
 hils_status check_device_errors() {
+    if (summary_error_flags(true) != 0)
+        return fail(HILS_ERR_TIMEOUT, "hils_check: a summary tile's copy did not complete within its wait budget; "
+                    "that call's summaries are invalid");
     if (select_tc_error_flags(true) != 0)
         return fail(HILS_ERR_TIMEOUT, "hils_check: a tensor-core selection tile's wait expired; that call's ids are "
                     "invalid");

@@ -1,5 +1,7 @@
 // Stage (a): landmark chunk summaries, "Hierarchical Sparse Attention Done Right" Eq. 8 (Prop. 3.1).
 //
+// This file is the general form (fp32 or bf16, any d and S); bf16 with d 128, S 64 and G <= 8 runs the
+// streamed tensor-core kernel of summary_mma.cu instead.
 // One CTA per (batch b, KV group g, chunk c). The chunk's S keys are read from HBM once into shared
 // memory (fp32) and reused by the G query heads of the group, one warp per head:
 //   u_j = tau * q'_{h,c} . k_j,  p = softmax(u),  k'_{h,c} = sum_j p_j k_j,  b'_{h,c} = LSE(u) - sum_j p_j u_j
@@ -84,9 +86,15 @@ summary_kernel(Dims D, const T *__restrict__ k, const T *__restrict__ q_land, in
 
 }  // namespace
 
+bool summary_mma_supported(const Dims &D, int dtype, const void *k, const void *q_land, const void *k_sum);
+cudaError_t launch_summary_mma(const Dims &D, const void *k, const void *q_land, int c_begin, int c_end,
+                               void *k_sum, float *b_sum, cudaStream_t stream);
+
 cudaError_t launch_chunk_summary(const Dims &D, int dtype, const void *k, const void *q_land, int c_begin, int c_end,
                                  void *k_sum, float *b_sum, cudaStream_t stream) {
     if (c_end <= c_begin) return cudaSuccess;
+    if (summary_mma_supported(D, dtype, k, q_land, k_sum))
+        return launch_summary_mma(D, k, q_land, c_begin, c_end, k_sum, b_sum, stream);
     const size_t smem = sizeof(float) * ((size_t)D.S * (D.d + 1) + (size_t)D.G * D.d + (size_t)kSummaryWarps * D.S);
     dim3 grid(c_end - c_begin, D.Hkv, D.B);
     if (dtype == HILS_BF16) {
