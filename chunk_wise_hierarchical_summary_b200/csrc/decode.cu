@@ -21,6 +21,13 @@
 #include "tma.cuh"
 
 namespace hils {
+
+bool decode_attn_mma_supported(const Dims &D, int dtype, const void *q, const void *k, const void *v, int ntiles);
+cudaError_t launch_decode_attn_mma(const Dims &D, int n, int ntiles, const void *q, const void *k_cache,
+                                   const void *v_cache, const float *scores, const int *sel, float *partial,
+                                   unsigned int *counters, void *out, float *lse, cudaStream_t stream);
+unsigned int decode_attn_mma_error_flags(bool clear);
+
 namespace {
 
 constexpr int kSelThreads = 256;
@@ -66,7 +73,7 @@ DecodePlan make_plan(const Dims &D) {
     P.off_part = take((size_t)D.B * D.Hq * P.nslices * kScorePartsPerSliceHost * 2 * sizeof(float));
     P.off_list = take((size_t)bg * P.nparts * D.topk * sizeof(uint64_t));
     P.off_sel = take((size_t)bg * D.topk * sizeof(int));
-    P.off_attn = take((size_t)D.B * D.Hq * P.ntiles * (D.d + 2) * sizeof(float));
+    P.off_attn = take((size_t)D.B * D.Hq * P.ntiles * (D.d + 4) * sizeof(float));  // either attention form
     P.off_count = take((size_t)bg * sizeof(unsigned int));
     P.off_selcount = take((size_t)bg * sizeof(unsigned int));
     P.total = off;
@@ -681,6 +688,9 @@ cudaError_t launch_t(const Dims &D, const void *q, const void *q_hat, const void
     unsigned int *selcount = (unsigned int *)(w + P.off_selcount);
     decode_select_kernel<<<dim3(P.nparts, D.Hkv, D.B), kSelThreads, 0, stream>>>(D, P, scores, part, lists, selcount,
                                                                                  sel, idx_out);
+    if (decode_attn_mma_supported(D, sizeof(T) == 2 ? HILS_BF16 : HILS_FP32, q, k_cache, v_cache, P.ntiles))
+        return launch_decode_attn_mma(D, P.n, P.ntiles, q, k_cache, v_cache, scores, sel, partial, counters, out, lse,
+                                      stream);
     const size_t smem3 = 2 * (size_t)D.S * D.d * sizeof(T) +
                          sizeof(float) * ((size_t)D.G * D.S + 4 + (size_t)D.G * D.d * 3 / 2 + D.G + 4 +
                                           2 * (size_t)D.G * D.d);
@@ -706,9 +716,11 @@ bool decode_supported(const Dims &D) {
 }
 
 unsigned int decode_error_flags(bool clear) {
-    unsigned int v = 0;
-    cudaMemcpyFromSymbol(&v, g_decode_errors, sizeof(v));
-    if (clear && v) {
+    unsigned int v = decode_attn_mma_error_flags(clear);
+    unsigned int mine = 0;
+    cudaMemcpyFromSymbol(&mine, g_decode_errors, sizeof(mine));
+    v |= mine;
+    if (clear && mine) {
         const unsigned int zero = 0;
         cudaMemcpyToSymbol(g_decode_errors, &zero, sizeof(zero));
     }

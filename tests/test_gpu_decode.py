@@ -52,6 +52,10 @@ def check_groups(w, x, k_sum, b_sum, out, lse, idx, groups):
                recipe="needle", q_pos0=299, needles=0),
     W.Workload("dec_topk_over_cands", B=1, T=1, L=900, Hq=4, Hkv=2, d=128, S=64, topk=32, W=512, dtype="bf16",
                recipe="needle", q_pos0=899, needles=2),
+    W.Workload("dec_g8_ragged", B=2, T=1, L=5000, Hq=16, Hkv=2, d=128, S=64, topk=12, W=300, dtype="bf16",
+               recipe="needle", q_pos0=4999, needles=5),
+    W.Workload("dec_g1", B=1, T=1, L=3000, Hq=3, Hkv=3, d=128, S=64, topk=8, W=200, dtype="bf16",
+               recipe="needle", q_pos0=2999, needles=3),
 ], ids=lambda w: w.name)
 def test_decode_shapes(w):
     x = W.decode_inputs(w, seed=1, device="cpu")
