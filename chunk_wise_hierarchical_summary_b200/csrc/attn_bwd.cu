@@ -8,6 +8,8 @@
 //   Eq. 8 backward: du_j = p_j (dk'.(k_j - k') - db' (log p_j + b')), dq'_c = tau sum_j du_j k_j,
 //                   dk_j += p_j dk' + tau du_j q'_c
 //
+// This file is the general form (CUDA cores, any dtype, d and S); bf16 with d 128, S 64, G <= 4 and
+// at most 128 chunks runs the tensor-core backward of attn_bwd_tc.cu instead.
 // Two deterministic kernels (no atomics):
 //   bwd_dq    query-major, one warp per (b, h, i): D, dq, dq^.
 //   bwd_dkdv  chunk-major, one CTA per (b, KV group, chunk c): every (query, head) touching the chunk
@@ -17,6 +19,14 @@
 #include "internal.h"
 
 namespace hils {
+
+bool attn_bwd_tc_supported(const Dims &D, int dtype);
+size_t attn_bwd_tc_workspace(const Dims &D);
+cudaError_t launch_attn_bwd_tc(const Dims &D, const void *q, const void *k, const void *v, const void *q_hat,
+                               const void *q_land, const void *k_sum, const float *b_sum, const int *idx,
+                               const void *out, const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                               void *dq_hat, void *dq_land, void *ws, cudaStream_t stream);
+
 namespace {
 
 constexpr int kDqWarps = 4;
@@ -394,7 +404,10 @@ cudaError_t launch_t(const Dims &D, const void *q, const void *k, const void *v,
 
 }  // namespace
 
-size_t bwd_workspace_bytes(const Dims &D) { return ((size_t)D.B * D.Hq * D.T * sizeof(float) + 255) & ~(size_t)255; }
+size_t bwd_workspace_bytes(const Dims &D, int dtype) {
+    if (attn_bwd_tc_supported(D, dtype)) return attn_bwd_tc_workspace(D);
+    return ((size_t)D.B * D.Hq * D.T * sizeof(float) + 255) & ~(size_t)255;
+}
 
 size_t bwd_smem_bytes(const Dims &D) { return dkv_layout(D.S, D.d, D.G).total; }
 
@@ -402,6 +415,9 @@ cudaError_t launch_attn_bwd(const Dims &D, int dtype, const void *q, const void 
                             const void *q_land, const void *k_sum, const float *b_sum, const int *idx,
                             const void *out, const float *lse, const void *dout, void *dq, void *dk, void *dv,
                             void *dq_hat, void *dq_land, void *ws, cudaStream_t stream) {
+    if (attn_bwd_tc_supported(D, dtype))
+        return launch_attn_bwd_tc(D, q, k, v, q_hat, q_land, k_sum, b_sum, idx, out, lse, dout, dq, dk, dv, dq_hat,
+                                  dq_land, ws, stream);
     if (dtype == HILS_BF16)
         return launch_t<__nv_bfloat16>(D, q, k, v, q_hat, q_land, k_sum, b_sum, idx, out, lse, dout, dq, dk, dv,
                                        dq_hat, dq_land, ws, stream);

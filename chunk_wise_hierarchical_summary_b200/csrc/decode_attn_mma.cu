@@ -19,6 +19,7 @@
 #include <algorithm>
 
 #include "internal.h"
+#include "mma_sync.cuh"
 #include "tcgen05.cuh"
 
 namespace hils {
@@ -40,44 +41,6 @@ constexpr int kPartStride = 132;  // floats per (head, split) partial: M, l, 2 p
 
 __device__ unsigned int g_decode_attn_errors = 0;
 
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void bar_consumers() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
-}
-__device__ __forceinline__ bool bar_consumers_any(bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.or.pred p, 1, %2, q;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "n"(kConsumerWarps * 32)
-        : "memory");
-    return r != 0;
-}
-__device__ __forceinline__ uint32_t ld_u32(const void *p) { return *reinterpret_cast<const uint32_t *>(p); }
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
 
 struct Tile {
     int j0, jn, c;  // first token, valid tokens, chunk id (-1: window tile)
@@ -202,7 +165,7 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
                 red_m[warp][2 * t4] = m0;
                 red_m[warp][2 * t4 + 1] = m1;
             }
-            if (bar_consumers_any(!got)) {
+            if (bar_group_any<kConsumerWarps * 32>(!got)) {
                 ok = false;
                 break;
             }
@@ -212,7 +175,7 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
                 mt0 = fmaxf(mt0, red_m[w][2 * t4]);
                 mt1 = fmaxf(mt1, red_m[w][2 * t4 + 1]);
             }
-            const float e00 = ex2(s00 - mt0), e01 = ex2(s01 - mt1), e10 = ex2(s10 - mt0), e11 = ex2(s11 - mt1);
+            const float e00 = ex2_approx(s00 - mt0), e01 = ex2_approx(s01 - mt1), e10 = ex2_approx(s10 - mt0), e11 = ex2_approx(s11 - mt1);
             float z0 = e00 + e10, z1 = e01 + e11;
 #pragma unroll
             for (int x = 4; x < 32; x <<= 1) {
@@ -223,7 +186,7 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
                 red_z[warp][2 * t4] = z0;
                 red_z[warp][2 * t4 + 1] = z1;
             }
-            bar_consumers();
+            bar_group<kConsumerWarps * 32>();
             float Z0 = 0.f, Z1 = 0.f;
 #pragma unroll
             for (int w = 0; w < kConsumerWarps; ++w) {
@@ -233,8 +196,8 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
             const float A0 = tl.c >= 0 ? sh0 - __log2f(Z0) : mt0;
             const float A1 = tl.c >= 0 ? sh1 - __log2f(Z1) : mt1;
             const float N0 = fmaxf(M0, A0), N1 = fmaxf(M1, A1);
-            const float fo0 = ex2(M0 - N0), fo1 = ex2(M1 - N1);  // 0 while M is still -inf
-            const float fn0 = ex2(A0 - N0), fn1 = ex2(A1 - N1);
+            const float fo0 = ex2_approx(M0 - N0), fo1 = ex2_approx(M1 - N1);  // 0 while M is still -inf
+            const float fn0 = ex2_approx(A0 - N0), fn1 = ex2_approx(A1 - N1);
             M0 = N0;
             M1 = N1;
             l0 = l0 * fo0 + Z0 * fn0;
@@ -257,7 +220,7 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
                     p_lo[hh[e] * kPStride + jj[e]] = __float2bfloat16_rn(pv[e] - __bfloat162float(hi));
                 }
             }
-            bar_consumers();
+            bar_group<kConsumerWarps * 32>();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 const int j0 = 16 * kk;
@@ -326,7 +289,7 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
         for (int s = 0; s < nsplit; ++s) {
             const float ms = __ldcg(ph + (size_t)s * kPartStride);
             if (ms == -INFINITY) continue;  // a CTA with no tiles
-            const float r = ex2(ms - M);
+            const float r = ex2_approx(ms - M);
             Z += __ldcg(ph + (size_t)s * kPartStride + 1) * r;
             const float4 v4 = __ldcg(reinterpret_cast<const float4 *>(ph + (size_t)s * kPartStride + 4) + lane);
             acc[0] = fmaf(v4.x, r, acc[0]);

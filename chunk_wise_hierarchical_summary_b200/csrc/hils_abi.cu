@@ -27,6 +27,7 @@ cudaError_t launch_select_tc(const Dims &D, const void *q_hat, const void *k_sum
                              float *gap, cudaStream_t stream);
 unsigned int select_tc_error_flags(bool clear);
 unsigned int summary_error_flags(bool clear);
+unsigned int attn_bwd_tc_error_flags(bool clear);
 
 namespace {
 
@@ -105,6 +106,9 @@ hils_status check_device_errors() {
     if (attn_tc_error_flags(true) != 0)
         return fail(HILS_ERR_TIMEOUT, "hils_check: a tensor-core attention tile's wait expired; that call's output "
                     "is invalid");
+    if (attn_bwd_tc_error_flags(true) != 0)
+        return fail(HILS_ERR_TIMEOUT, "hils_check: a tensor-core backward tile's wait expired; that call's "
+                    "gradients are invalid");
     if (decode_error_flags(true) != 0)
         return fail(HILS_ERR_TIMEOUT, "hils_check: a decode tile's bulk copy did not complete within its wait "
                     "budget; that call's output is invalid");
@@ -141,7 +145,7 @@ size_t hils_workspace_size(const hils_params *p, int op) {
         case HILS_OP_SELECT: return 0;
         case HILS_OP_ATTN_FWD: return attn_fwd_tc_supported(D, p->dtype) ? attn_fwd_tc_workspace(D) : 0;
         case HILS_OP_DECODE: return decode_workspace_bytes(D);
-        case HILS_OP_ATTN_BWD: return bwd_workspace_bytes(D);
+        case HILS_OP_ATTN_BWD: return bwd_workspace_bytes(D, p->dtype);
         default: return (size_t)-1;
     }
 }
@@ -280,7 +284,7 @@ hils_status hils_attn_bwd(const hils_params *p, const void *q, const void *k, co
     if (D.Hkv > 65535) return fail(HILS_ERR_UNSUPPORTED, "%s: Hkv must be <= 65535", fn);
     if (bwd_smem_bytes(D) > kMaxSmem)
         return fail(HILS_ERR_UNSUPPORTED, "%s: S=%d, d=%d, G=%d exceed one CTA's shared memory", fn, D.S, D.d, D.G);
-    st = check_ws(fn, workspace, workspace_bytes, bwd_workspace_bytes(D));
+    st = check_ws(fn, workspace, workspace_bytes, bwd_workspace_bytes(D, p->dtype));
     if (st != HILS_OK) return st;
     return cuda_status(launch_attn_bwd(D, p->dtype, q, k, v, q_hat, q_land, k_sum, b_sum, idx, out, lse, dout, dq, dk,
                                        dv, dq_hat, dq_land, workspace, (cudaStream_t)stream),

@@ -28,7 +28,7 @@ cudaError_t launch_decode(const Dims &D, int dtype, const void *q, const void *q
 // Device-side error words (bit set when a bounded wait expired); reading with clear resets them.
 unsigned int decode_error_flags(bool clear);
 
-size_t bwd_workspace_bytes(const Dims &D);
+size_t bwd_workspace_bytes(const Dims &D, int dtype);
 cudaError_t launch_attn_bwd(const Dims &D, int dtype, const void *q, const void *k, const void *v, const void *q_hat,
                             const void *q_land, const void *k_sum, const float *b_sum, const int *idx,
                             const void *out, const float *lse, const void *dout, void *dq, void *dk, void *dv,

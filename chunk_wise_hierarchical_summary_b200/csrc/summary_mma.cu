@@ -16,6 +16,7 @@
 #include <algorithm>
 
 #include "internal.h"
+#include "mma_sync.cuh"
 #include "tcgen05.cuh"
 
 namespace hils {
@@ -36,41 +37,6 @@ constexpr int kPStride = 72;             // bf16 elements per row of p (64 + 8 p
 
 __device__ unsigned int g_summary_errors = 0;
 
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-// c += a (16x16, row) * b (16x8, col), bf16 inputs, fp32 accumulators.
-__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void bar_consumers() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
-}
-// Barrier over the consumer warps that also returns, to every one of them, whether any passed `pred`.
-__device__ __forceinline__ bool bar_consumers_any(bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.or.pred p, 1, %2, q;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "n"(kConsumerWarps * 32)
-        : "memory");
-    return r != 0;
-}
-__device__ __forceinline__ uint32_t ld_u32(const void *p) { return *reinterpret_cast<const uint32_t *>(p); }
 
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 summary_mma_kernel(const __grid_constant__ CUtensorMap kmap, Dims D, const __nv_bfloat16 *__restrict__ q_land,
@@ -157,7 +123,7 @@ summary_mma_kernel(const __grid_constant__ CUtensorMap kmap, Dims D, const __nv_
                 red_m[warp][2 * t4] = m0;
                 red_m[warp][2 * t4 + 1] = m1;
             }
-            if (bar_consumers_any(!got)) {  // uniform across the consumer warps
+            if (bar_group_any<kConsumerWarps * 32>(!got)) {  // uniform across the consumer warps
                 ok = false;
                 break;
             }
@@ -184,7 +150,7 @@ summary_mma_kernel(const __grid_constant__ CUtensorMap kmap, Dims D, const __nv_
                 red_e[warp][2 * t4] = eu0;
                 red_e[warp][2 * t4 + 1] = eu1;
             }
-            bar_consumers();
+            bar_group<kConsumerWarps * 32>();
             float Z0 = 0.f, Z1 = 0.f, EU0 = 0.f, EU1 = 0.f;
 #pragma unroll
             for (int w = 0; w < kConsumerWarps; ++w) {
@@ -206,7 +172,7 @@ summary_mma_kernel(const __grid_constant__ CUtensorMap kmap, Dims D, const __nv_
                     p_lo[hh[e] * kPStride + jj[e]] = __float2bfloat16_rn(pv[e] - __bfloat162float(hi));
                 }
             }
-            bar_consumers();
+            bar_group<kConsumerWarps * 32>();
             // k'^T for columns 32w..32w+31 (two 16-row tiles), heads 0..7
             float o[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
@@ -235,7 +201,7 @@ summary_mma_kernel(const __grid_constant__ CUtensorMap kmap, Dims D, const __nv_
                 outs[2 * t4][dd + 8] = __float2bfloat16_rn(o[mt][2]);
                 outs[2 * t4 + 1][dd + 8] = __float2bfloat16_rn(o[mt][3]);
             }
-            bar_consumers();
+            bar_group<kConsumerWarps * 32>();
             const int c = c_begin + (int)(u % nc);
             const long long rest = u / nc;
             const int g = (int)(rest % D.Hkv), b = (int)(rest / D.Hkv);

@@ -11,6 +11,10 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running (full-size workloads)")
+    # a library older than its sources is rebuilt before anything loads it (no-op when up to date)
+    from chunk_wise_hierarchical_summary_b200 import build
+
+    build.build()
 
 
 @pytest.fixture(scope="session")

@@ -50,6 +50,10 @@ def run_bwd(w, seed=0):
                recipe="scaled"),
     W.Workload("bwd_fp32_d128_S16", B=1, T=333, L=333, Hq=2, Hkv=1, d=128, S=16, topk=5, W=20, dtype="fp32",
                recipe="tiny"),
+    W.Workload("bwd_bf16_g2_nc15", B=1, T=1000, L=1000, Hq=4, Hkv=2, d=128, S=64, topk=4, W=128, dtype="bf16",
+               recipe="scaled"),
+    W.Workload("bwd_bf16_g1", B=1, T=900, L=900, Hq=2, Hkv=2, d=128, S=64, topk=5, W=200, dtype="bf16",
+               recipe="scaled"),
 ], ids=lambda w: w.name)
 def test_backward_shapes(w):
     run_bwd(w)
