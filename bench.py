@@ -486,14 +486,15 @@ def run_reference(args, dist):
 def profile_case(args):
     """`--profile STAGE`: `args.steps` untimed launches of one stage on its workload, for ncu captures of
     one kernel (select it with ncu's -k / -s / -c). Prints no bench line. The summary case runs on a
-    128K-token cache (B1; 256 MiB of keys, above L2), the decode case on the 512K decode workload."""
+    128K-token cache (B1; 256 MiB of keys, above L2), the decode case on a 512K-token cache at B1 (2 GiB of
+    K and V: the decode workload's per-sequence shape with a footprint a profiler can save and restore)."""
     import chunk_wise_hierarchical_summary_b200.hils as H
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     st = args.profile
     if st in ("summary", "decode"):
-        w = W.DECODE_BF16 if st == "decode" else W.decode_sweep(131072)
+        w = W.decode_sweep(524288) if st == "decode" else W.decode_sweep(131072)
         x = W.decode_inputs(w, seed=2000, device=dev)
         k_sum, b_sum = H.chunk_summary(x["k_cache"], x["q_land"], w.S)
         if st == "summary":
