@@ -1,22 +1,22 @@
 // Single-token decode over a long KV cache: stages (b)-(d) for one query at position L-1
 // ("Hierarchical Sparse Attention Done Right", Eq. 7, Sec. 3 RQ1, Sec. 4 "GQA", Eq. 10).
 //
-// Three launches; one query row per head means no dense contraction, so these are HBM-streaming
-// CUDA-core kernels:
-//  1. score    grid (slices, Hq, B): each CTA pulls one 128-candidate slice of a head's summaries
-//              (32 KiB at d 128 bf16) into shared memory with a single TMA bulk copy, then computes
-//              s^_{h,c} = tau q^_h . k'_{h,c} + b'_{h,c} into a score buffer, plus the slice's partial
-//              (max, sum exp).
-//  2. select   grid (Hkv, B). Per-head LSE from the partials; group score g_c = max_h (s^_{h,c} - LSE_h)
-//              as order-preserving 32-bit keys; an MSB-first radix select (four byte passes, warp-
-//              aggregated shared-memory histogram) finds the k-th largest key; an ordered compaction
-//              keeps every larger key and the lowest-id equal keys (the tie rule); one warp sorts
-//              those k entries and writes the ids ascending.
-//  3. attend   grid (tiles, Hkv, B): one S-token tile (a selected chunk or a window tile) per CTA; K
-//              and V staged by TMA bulk copies; all G heads; a partial (max, sum, acc[d]) of the online
-//              softmax over adjusted logits (a chunk token carries s_j - L_c + s^_c, s^_c read from the
-//              score buffer). The last CTA of each (b, KV group) to finish (an atomic counter, no
-//              waiting) merges the group's partials into out and lse.
+// Three launches (plus one memset of the counters):
+//  1. score    persistent, one CTA per SM: a producer lane keeps a ring of bulk copies of 128-candidate
+//              summary slices (32 KiB at d 128 bf16) in flight; consumer warps compute
+//              s^_{h,c} = tau q^_h . k'_{h,c} + b'_{h,c} into a score buffer plus per-warp partials
+//              (max, sum exp) of each slice. This launch streams the decode step's dominant bytes.
+//  2. select   per (b, KV group): per-head LSE folded from the partials, group score
+//              g_c = max_h (s^_{h,c} - LSE_h) as 64-bit keys (score desc, chunk id asc), top-k. For
+//              topk <= 32 and G <= 8 one CTA per group: each warp sorts batches of 256 keys in registers
+//              and merges their best 32 into a running top-32, then the warps' lists are reduced in
+//              the CTA. Otherwise several CTAs per group keep their part's top-k and the last CTA to
+//              finish (atomic counter, no waiting) merges them.
+//  3. attend   bf16 d 128 S 64 G <= 8: decode_attn_mma.cu (split-K CTAs over the group's tiles,
+//              warp-level MMAs, online Eq. 10 merge). Otherwise here: one S-token tile (a selected
+//              chunk or a window tile) per CTA, K and V staged by bulk copies, all G heads, a partial
+//              (max, sum, acc[d]) of the online softmax over adjusted logits (a chunk token carries
+//              s_j - L_c + s^_c); the last CTA of each (b, KV group) merges the partials into out, lse.
 #include "internal.h"
 #include "tma.cuh"
 
@@ -459,6 +459,246 @@ decode_select_kernel(Dims D, DecodePlan P, const float *__restrict__ scores, con
     }
 }
 
+// Lane l receives element l of a warp-sorted sequence of 32*NPL keys (element e at lane e / NPL,
+// slot e % NPL): the 32 smallest, one per lane, ascending.
+template <int NPL>
+__device__ __forceinline__ uint64_t warp_first32(const uint64_t (&v)[NPL]) {
+    const int lane = threadIdx.x & 31;
+    uint64_t mine = ~0ull;
+#pragma unroll
+    for (int s = 0; s < NPL; ++s) {
+        const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)v[s], lane / NPL);
+        const uint32_t hi = __shfl_sync(0xffffffffu, (uint32_t)(v[s] >> 32), lane / NPL);
+        if (lane % NPL == s) mine = ((uint64_t)hi << 32) | lo;
+    }
+    return mine;
+}
+
+// The 32 smallest of two ascending one-per-lane lists, ascending: min(a_l, b_{31-l}) is bitonic, then a
+// bitonic merge.
+__device__ __forceinline__ uint64_t warp_merge_lowest32(uint64_t a, uint64_t b) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t blo = __shfl_sync(0xffffffffu, (uint32_t)b, 31 - lane);
+    const uint32_t bhi = __shfl_sync(0xffffffffu, (uint32_t)(b >> 32), 31 - lane);
+    const uint64_t br = ((uint64_t)bhi << 32) | blo;
+    uint64_t v = a < br ? a : br;
+#pragma unroll
+    for (int st = 16; st > 0; st >>= 1) {
+        const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, st);
+        const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), st);
+        const uint64_t p = ((uint64_t)hi << 32) | lo;
+        v = ((lane & st) == 0) ? (v < p ? v : p) : (v > p ? v : p);
+    }
+    return v;
+}
+
+// Slow path of the single-CTA selection, kept out of line so that its code is fetched only when used
+// (massively tied scores overflow the survivor buffer): every warp keeps a running top-32 of its
+// candidates, merged in registers batch by batch, and the CTA reduces the warps' lists. Returns the 32
+// smallest keys, ascending, to warp 0 (one per lane).
+template <int GM>
+__device__ __noinline__ uint64_t select_tied_fallback(const float *__restrict__ sc0, int G, int n, int rounds,
+                                                      const float (&L)[8], uint64_t *keys) {
+    constexpr int kPer = 64 / GM, kRound = 512 * kPer;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    uint64_t best = ~0ull;
+    for (int r = 0; r < rounds; ++r) {
+        for (int h = 0; h < kPer / 8; ++h) {
+            uint64_t kv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int c = r * kRound + warp * (32 * kPer) + (h * 8 + i) * 32 + lane;
+                float gv = -INFINITY;
+                for (int hh = 0; hh < G; ++hh) gv = fmaxf(gv, (c < n ? sc0[(size_t)hh * n + c] : -INFINITY) - L[hh]);
+                kv[i] = (c < n) ? desc_value_key(gv, (uint32_t)c) : ~0ull;
+            }
+            warp_bitonic_sort<8>(kv);
+            best = warp_merge_lowest32(best, warp_first32<8>(kv));
+        }
+    }
+    __syncthreads();
+    keys[warp * 32 + lane] = best;
+    for (int span = 1; span < nwarps; span <<= 1) {
+        __syncthreads();
+        uint64_t m = ~0ull;
+        const bool act = (warp % (2 * span)) == 0 && warp + span < nwarps;
+        if (act) m = warp_merge_lowest32(keys[warp * 32 + lane], keys[(warp + span) * 32 + lane]);
+        __syncthreads();
+        if (act) keys[warp * 32 + lane] = m;
+    }
+    __syncthreads();
+    return warp == 0 ? keys[lane] : ~0ull;
+}
+
+// Single-CTA selection of one (b, KV group) for topk <= 32 and G <= 8. Keys as in the multi-CTA form
+// (group score desc, chunk id asc; all distinct), so the same ids.
+//  1. per-head LSE folded from the score kernel's slice partials; group keys of every candidate, and
+//     each thread's best (smallest) key;
+//  2. bound: the 32nd smallest of the 512 per-thread best keys. At least 32 candidates (one per
+//     thread holding those keys) are at or below it, so the 32 smallest keys overall all are too;
+//  3. the candidates at or below the bound (about 32-50 on any non-degenerate scores) are compacted
+//     into shared memory and sorted by one warp; their first k are the selection.
+// When the survivors overflow the buffer (massively tied scores) select_tied_fallback takes over.
+// GM: heads held per candidate (4 or 8); a thread keeps 64 raw scores in flight per round.
+constexpr int kSelWThreads = 512;
+constexpr int kSelWCap = 128;  // survivor buffer (sorted by one warp, 4 keys per lane)
+
+template <int GM>
+__global__ void __launch_bounds__(kSelWThreads)
+decode_select_warp_kernel(Dims D, DecodePlan P, const float *__restrict__ scores, const float *__restrict__ part,
+                          int *__restrict__ sel, int *__restrict__ idx_out) {
+    __shared__ float lse[8];
+    __shared__ __align__(8) uint64_t keys[kSelWThreads];
+    __shared__ __align__(8) uint64_t surv[kSelWCap];
+    __shared__ uint64_t s_bound;
+    __shared__ int s_count;
+    const int g = blockIdx.x, b = blockIdx.y;
+    const int G = D.G, K = D.topk, n = P.n;
+    const size_t bg = (size_t)b * D.Hkv + g;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = kSelWThreads / 32;
+    int *out = sel + bg * K;
+    int *out2 = idx_out ? idx_out + bg * K : nullptr;
+    if (n == 0) {
+        for (int t = tid; t < K; t += blockDim.x) {
+            out[t] = -1;
+            if (out2) out2[t] = -1;
+        }
+        return;
+    }
+    const float *sc0 = scores + ((size_t)b * D.Hq + g * G) * n;
+    constexpr int kSelWPer = 64 / GM;                     // candidates per thread per round
+    constexpr int kSelWRound = kSelWThreads * kSelWPer;
+    const int rounds = (n + kSelWRound - 1) / kSelWRound;
+    // candidate of (round r, slot i) for this thread: coalesced across the warp
+    auto cand = [&](int r, int i) { return r * kSelWRound + warp * (32 * kSelWPer) + i * 32 + lane; };
+    float raw[GM][kSelWPer];
+    auto load_round = [&](int r) {
+#pragma unroll
+        for (int hh = 0; hh < GM; ++hh)
+#pragma unroll
+            for (int i = 0; i < kSelWPer; ++i) {
+                const int c = cand(r, i);
+                raw[hh][i] = (hh < G && c < n) ? sc0[(size_t)hh * n + c] : -INFINITY;
+            }
+    };
+    load_round(0);  // in flight during the LSE fold
+    if (tid == 0) s_count = 0;
+    if (warp < G) {
+        const int hh = warp;
+        const int np = P.nslices * kScorePartsPerSliceHost;
+        const float2 *ph = reinterpret_cast<const float2 *>(part + ((size_t)b * D.Hq + g * G + hh) * np * 2);
+        float M = -INFINITY, Z = 0.f;
+        for (int s0 = 0; s0 < np; s0 += 32 * 8) {
+            float2 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int si = s0 + u * 32 + lane;
+                v[u] = (si < np) ? ph[si] : make_float2(-INFINITY, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (v[u].x > M) {
+                    Z = Z * __expf(M - v[u].x) + v[u].y;
+                    M = v[u].x;
+                } else if (v[u].x > -INFINITY) {
+                    Z += v[u].y * __expf(v[u].x - M);
+                }
+            }
+        }
+        const float MM = warp_max(M);
+        Z = (M > -INFINITY) ? Z * __expf(M - MM) : 0.f;
+        Z = warp_sum(Z);
+        if (lane == 0) lse[hh] = MM + logf(Z);
+    }
+    __syncthreads();
+    float L[8];
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh) L[hh] = hh < G ? lse[hh] : 0.f;
+    auto key_of = [&](int r, int i) -> uint64_t {
+        const int c = cand(r, i);
+        float gv = -INFINITY;
+#pragma unroll
+        for (int hh = 0; hh < GM; ++hh)
+            if (hh < G) gv = fmaxf(gv, raw[hh][i] - L[hh]);
+        return (c < n) ? desc_value_key(gv, (uint32_t)c) : ~0ull;
+    };
+
+    // 1. each thread's best key
+    uint64_t mine = ~0ull;
+    for (int r = 0; r < rounds; ++r) {
+        if (r > 0) load_round(r);
+#pragma unroll
+        for (int i = 0; i < kSelWPer; ++i) {
+            const uint64_t k = key_of(r, i);
+            mine = k < mine ? k : mine;
+        }
+    }
+    // 2. the 32nd smallest of the per-thread best keys: sort within each warp, then merge the warps'
+    //    ascending lists pairwise
+    {
+        uint64_t one[1] = {mine};
+        warp_bitonic_sort<1>(one);
+        keys[warp * 32 + lane] = one[0];
+    }
+    for (int span = 1; span < nwarps; span <<= 1) {
+        __syncthreads();
+        uint64_t m = ~0ull;
+        const bool act = (warp % (2 * span)) == 0 && warp + span < nwarps;
+        if (act) m = warp_merge_lowest32(keys[warp * 32 + lane], keys[(warp + span) * 32 + lane]);
+        __syncthreads();
+        if (act) keys[warp * 32 + lane] = m;
+    }
+    __syncthreads();
+    if (tid == 0) s_bound = keys[31];
+    __syncthreads();
+    const uint64_t bound = s_bound;
+    // 3. compact the candidates at or below the bound (scores reloaded when they did not fit one round)
+    for (int r = 0; r < rounds; ++r) {
+        if (rounds > 1) load_round(r);
+#pragma unroll
+        for (int i = 0; i < kSelWPer; ++i) {
+            const uint64_t k = key_of(r, i);
+            const bool take = k <= bound && k != ~0ull;  // (padding slots never qualify)
+            const unsigned m = __ballot_sync(0xffffffffu, take);
+            if (m) {
+                int base = 0;
+                if (lane == 0) base = atomicAdd(&s_count, __popc(m));
+                base = __shfl_sync(0xffffffffu, base, 0);
+                const int at = base + __popc(m & ((1u << lane) - 1));
+                if (take && at < kSelWCap) surv[at] = k;
+            }
+        }
+    }
+    __syncthreads();
+    const int count = s_count;
+    uint64_t top = ~0ull;  // warp 0: the selection's keys, ascending, one per lane
+    if (count <= kSelWCap) {
+        if (warp == 0) {
+            uint64_t kv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int e = lane * 4 + i;
+                kv[i] = e < count ? surv[e] : ~0ull;
+            }
+            warp_bitonic_sort<4>(kv);
+            top = warp_first32<4>(kv);
+        }
+    } else {
+        top = select_tied_fallback<GM>(sc0, G, n, rounds, L, keys);
+    }
+    if (warp == 0) {
+        // the selected ids (first min(K, n) keys), written ascending, -1 padded
+        const int kk = min(K, n);
+        uint64_t ids[1] = {(lane < kk && top != ~0ull) ? (uint64_t)desc_key_index(top) : ~0ull};
+        warp_bitonic_sort<1>(ids);
+        if (lane < K) {
+            const int v = ids[0] == ~0ull ? -1 : (int)ids[0];
+            out[lane] = v;
+            if (out2) out2[lane] = v;
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------- 3. attend (+ combine)
 
 template <typename T, int DPL>
@@ -686,8 +926,13 @@ cudaError_t launch_t(const Dims &D, const void *q, const void *q_hat, const void
                                                            part);
     }
     unsigned int *selcount = (unsigned int *)(w + P.off_selcount);
-    decode_select_kernel<<<dim3(P.nparts, D.Hkv, D.B), kSelThreads, 0, stream>>>(D, P, scores, part, lists, selcount,
-                                                                                 sel, idx_out);
+    if (D.topk <= 32 && D.G <= 4)
+        decode_select_warp_kernel<4><<<dim3(D.Hkv, D.B), kSelWThreads, 0, stream>>>(D, P, scores, part, sel, idx_out);
+    else if (D.topk <= 32 && D.G <= 8)
+        decode_select_warp_kernel<8><<<dim3(D.Hkv, D.B), kSelWThreads, 0, stream>>>(D, P, scores, part, sel, idx_out);
+    else
+        decode_select_kernel<<<dim3(P.nparts, D.Hkv, D.B), kSelThreads, 0, stream>>>(D, P, scores, part, lists,
+                                                                                     selcount, sel, idx_out);
     if (decode_attn_mma_supported(D, sizeof(T) == 2 ? HILS_BF16 : HILS_FP32, q, k_cache, v_cache, P.ntiles))
         return launch_decode_attn_mma(D, P.n, P.ntiles, q, k_cache, v_cache, scores, sel, partial, counters, out, lse,
                                       stream);

@@ -135,18 +135,20 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
                 }
             }
             float *dst_s = ws_shat + (((size_t)b * D.Hq + g * G + hh) * D.T + i) * K;
+            // The operand stages are dead once every MMA has completed: each thread copies a 32-column
+            // block of its row into a private shared-memory row (stride 33 floats, conflict-free) and
+            // reads the selected columns back by index.
+            float *row32 = reinterpret_cast<float *>(base) + (size_t)tid * 33;
             int u = 0;
 #pragma unroll 1
             for (int t = 0; t < 4; ++t) {
                 float v[32];
                 tmem_ld32(lane_base + hh * 128 + 32 * t, v);
                 tmem_wait_ld();
-                while (u < ns && cl[u] < 32 * t + 32) {
-                    const int e0 = cl[u] - 32 * t;
-                    float val = 0.f;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) val = (e == e0) ? v[e] : val;
-                    dst_s[u] = fmaf(D.tau, val, bs[hh][cl[u]]);
+                for (int e = 0; e < 32; ++e) row32[e] = v[e];
+                while (u < ns && cl[u] < 32 * t + 32) {
+                    dst_s[u] = fmaf(D.tau, row32[cl[u] - 32 * t], bs[hh][cl[u]]);
                     ++u;
                 }
             }

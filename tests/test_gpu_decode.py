@@ -108,3 +108,30 @@ def test_decode_sweep_sampled(L):
                              window=w.W, return_idx=True)
     torch.cuda.synchronize()
     check_groups(w, x, k_sum, b_sum, out, lse, idx, [(0, 0), (0, 6)])
+
+
+def test_decode_select_periodic_scores():
+    """Scores boosted on every 32nd candidate: one lane of every warp of the single-CTA selection holds
+    all the winners, so the candidates at or below the per-thread bound (about 200 here) overflow the
+    survivor buffer and the out-of-line running-top-32 path decides. Ids must still equal the oracle's
+    selection on the same summaries, and the attention must match the oracle's with those ids."""
+    w = W.Workload("dec_periodic", B=1, T=1, L=400000, Hq=4, Hkv=1, d=128, S=64, topk=32, W=512, dtype="bf16",
+                   recipe="needle", q_pos0=399999, needles=0)
+    x = W.decode_inputs(w, seed=5, device="cpu")
+    g = torch.Generator().manual_seed(11)
+    k_sum = (torch.randn((1, w.Hq, w.Nc, w.d), generator=g) * 0.5).to(torch.bfloat16)  # spread: no near ties
+    b_sum = torch.zeros((1, w.Hq, w.Nc), dtype=torch.float32)
+    b_sum[:, :, ::32] = 8.0
+    xd = {n: t.cuda() for n, t in x.items()}
+    out, lse, idx = H.decode(xd["q"], xd["q_hat"], xd["k_cache"], xd["v_cache"], k_sum.cuda(), b_sum.cuda(), S=w.S,
+                             topk=w.topk, window=w.W, return_idx=True)
+    g1 = Geometry(B=1, T=1, L=w.L, Hq=w.G, Hkv=1, d=w.d, S=w.S, topk=w.topk, W=w.W, q_pos0=w.L - 1)
+    rk, rb = np64(k_sum), np64(b_sum)
+    qh = np64(x["q_hat"])
+    ridx, rgap = oracle.select_topk(g1, qh, rk, rb)
+    assert (np.asarray(ridx).reshape(-1) % 32 == 0).all()  # the boosted candidates win
+    near = check_idx(idx[:, :, None], ridx, rgap, "periodic idx")
+    assert not near.any()
+    ro, rl = oracle.attn_fwd(g1, np64(x["q"]), np64(x["k_cache"]), np64(x["v_cache"]), qh, rk, rb, ridx)
+    assert_close(out, ro, TOL["bf16"], "periodic out")
+    assert_close(lse, rl[..., 0], TOL["bf16"], "periodic lse")
