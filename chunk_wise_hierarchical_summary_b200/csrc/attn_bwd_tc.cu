@@ -164,7 +164,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
     __shared__ float lsh[128][kMaxK];  // per row: the matching s^ in log2 units
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = D.G, QT = 128 / G;
-    const int i0 = blockIdx.x * QT, g = blockIdx.y, b = blockIdx.z;
+    // late query tiles visit the most chunks: launch them first (short CTAs make the grid's tail)
+    const int i0 = (gridDim.x - 1 - blockIdx.x) * QT, g = blockIdx.y, b = blockIdx.z;
     const int S = D.S, K = D.topk;
     unsigned char *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     unsigned char *Qs = base, *DOs = base + kRowTile;

@@ -66,7 +66,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     __shared__ int s_ntiles;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = D.G, QT = 128 / G;
-    const int i0 = blockIdx.x * QT, g = blockIdx.y, b = blockIdx.z;
+    // Late query tiles visit the most chunks (every earlier candidate): launch them first so that the
+    // grid's tail is made of short CTAs.
+    const int i0 = (gridDim.x - 1 - blockIdx.x) * QT, g = blockIdx.y, b = blockIdx.z;
     const int S = D.S, K = D.topk;
     unsigned char *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     unsigned char *Qs = base;

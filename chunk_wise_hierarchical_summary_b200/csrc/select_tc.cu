@@ -170,30 +170,33 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
         return;
     }
 
-    // Phase 1: per-head log-partition over the row's candidates.
+    // Phase 1: per-head log-partition over the row's candidates, one 32-column block at a time (block
+    // max, then one rescale of the running sum per block).
     if (j < G) {
         const int hh = j;
         float m = -INFINITY, z = 0.f;
-#pragma unroll
+#pragma unroll 1
         for (int t = 0; t < 4; ++t) {
             float v[32];
             tmem_ld32(lane_base + hh * 128 + 32 * t, v);
             tmem_wait_ld();
+            float bm = -INFINITY;
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
                 const int c = 32 * t + e;
-                if (c < n_r) {
-                    const float sc = fmaf(D.tau, v[e], bs[hh][c]);
-                    if (sc > m) {
-                        z = z * __expf(m - sc) + 1.f;
-                        m = sc;
-                    } else {
-                        z += __expf(sc - m);
-                    }
-                }
+                v[e] = (c < n_r) ? fmaf(D.tau, v[e], bs[hh][c]) * kLog2e : -INFINITY;
+                bm = fmaxf(bm, v[e]);
+            }
+            if (bm > -INFINITY) {
+                const float mn = fmaxf(m, bm);
+                float zz = 0.f;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) zz += ex2_approx(v[e] - mn);
+                z = z * ex2_approx(m - mn) + zz;  // m = -inf at the first block: 2^-inf = 0
+                m = mn;
             }
         }
-        lse[hh][r] = (n_r > 0) ? m + logf(z) : 0.f;
+        lse[hh][r] = (n_r > 0) ? (m + log2f(z)) * kLn2 : 0.f;
     }
     tc_fence_before();
     __syncthreads();
@@ -237,9 +240,12 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
     }
     tc_fence_before();
     __syncthreads();  // every TMEM read done; operand tiles are dead: reuse them for the lists
-    uint64_t *lists = reinterpret_cast<uint64_t *>(base);  // [128 rows][4 blocks][K1MAX]
+    // [128 rows][4 blocks][K1MAX], rows padded by one key so that neighbouring rows' lists fall in
+    // different shared-memory banks
+    constexpr int kRowKeys = 4 * K1MAX + 1;
+    uint64_t *lists = reinterpret_cast<uint64_t *>(base);
 #pragma unroll
-    for (int t = 0; t < K1MAX; ++t) lists[((size_t)r * 4 + j) * K1MAX + t] = top[t];
+    for (int t = 0; t < K1MAX; ++t) lists[(size_t)r * kRowKeys + j * K1MAX + t] = top[t];
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
@@ -251,7 +257,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
         const int rr = tid, ii = i0 + rr;
         if (ii < D.T) {
             const int nn = window_left(D.q_pos0 + ii, D.W, D.S) / D.S;
-            const uint64_t *L = lists + (size_t)rr * 4 * K1MAX;
+            const uint64_t *L = lists + (size_t)rr * kRowKeys;
             int p0 = 0, p1 = 0, p2 = 0, p3 = 0;
             const int need = min(K + 1, nn);
             uint32_t ids[K1MAX];
@@ -314,11 +320,11 @@ cudaError_t launch_select_tc(const Dims &D, const void *q_hat, const void *k_sum
         return cudaErrorInvalidValue;
     dim3 grid((D.T + kRows - 1) / kRows, D.Hkv, D.B);
     if (D.topk <= 16) {
-        const size_t smem = 1024 + 2 * (size_t)kStageBytes;  // lists: 128 * 4 * 17 * 8 = 68 KiB fit in the stages
+        const size_t smem = 1024 + 2 * (size_t)kStageBytes;  // lists: 128 * 69 * 8 = 69 KiB fit in the stages
         cudaFuncSetAttribute(select_tc_kernel<17, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         select_tc_kernel<17, 0><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap, nullptr, nullptr);
     } else {
-        const size_t smem = 1024 + (size_t)kRows * 4 * 33 * 8;  // 132 KiB of lists > the two stages
+        const size_t smem = 1024 + (size_t)kRows * (4 * 33 + 1) * 8;  // 133 KiB of lists > the two stages
         cudaFuncSetAttribute(select_tc_kernel<33, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         select_tc_kernel<33, 0><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap, nullptr, nullptr);
     }
