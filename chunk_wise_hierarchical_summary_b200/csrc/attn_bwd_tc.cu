@@ -17,13 +17,15 @@
 //            chunks (as the forward): S = Q K^T and dP = dO V^T into TMEM, ds written over S in TMEM as
 //            bf16 pairs, dQ += ds K with ds read from TMEM. Two groups of four row warps take alternate
 //            tiles (rows need no running state in the backward). ds^ goes to a dense [rows x Nc] bf16
-//            matrix (zero where a chunk is not selected).
+//            matrix and beta = exp(s^ - lse) to a dense fp32 one (both zero where a chunk is not
+//            selected).
 //   dqhat    dq^ = tau ds^ K'  (warp per row, the head's summaries in shared memory)
 //   dksum    dk'^T, db' = the dense ds^ matrix contracted with q^ over the rows (mma.sync), split in
-//            four row ranges whose partials the next launch sums in a fixed order
+//            sixteen row ranges whose partials the next launch sums in a fixed order
 //   eq8      per (b, KV group, chunk): the Eq. 8 backward: dq' and an fp32 share of dk
 //   bkv      KV-major, tcgen05: CTA = one chunk (64 keys, K and V resident) streaming the query tiles
-//            that can reach it; S, dP as in bq, then P and ds (bf16, 128-byte swizzled, MN-major) in
+//            that can reach it (a row's beta for the chunk, lse and D fetched one tile ahead); S, dP as in
+//            bq, then P and ds (bf16, 128-byte swizzled, MN-major) in
 //            shared memory feed dV^T += dO^T P and dK^T += Q^T ds with both operands read transposed.
 #include <algorithm>
 
@@ -52,7 +54,7 @@ constexpr int kBitmapWords = 256;
 constexpr int kMaxK = 32;
 constexpr int kTcThreads = 320;  // producer, MMA issuer, two groups of four row warps
 constexpr int kBqStages = 3;
-constexpr int kDkSplit = 4;
+constexpr int kDkSplit = 16;  // row ranges of the dk'/db' reduction (partials summed in order)
 constexpr int kPartStride = 129;  // dk'(128) + db'(1) per (b, h, split, chunk)
 
 __device__ unsigned int g_bwd_tc_errors = 0;
@@ -76,13 +78,12 @@ __global__ void bwd_delta_kernel(const __nv_bfloat16 *__restrict__ out, const __
     if (l == 0 && r < rows) Dbuf[r] = s;
 }
 
-// One row's ds over a 64-token tile, shared by bq and bkv. s, dp: the row's raw logits (q . k) and
-// dout . v. On return s holds P_j and dp holds ds_j. kind: 1 selected chunk, 2 window, 0 neither.
-struct RowTile {
-    float dshat;  // ds^ of a selected chunk
-};
-__device__ __forceinline__ RowTile row_grad(float (&s)[64], float (&dp)[64], int kind, int lo, int hi, float sc2,
-                                            float lse2, float sh2, float Dr, bool warp_needs_mask) {
+// One row's ds over a 64-token tile, shared by bq and bkv, in two phases so that the dP load from TMEM
+// overlaps the exponentials. kind: 1 selected chunk, 2 window, 0 neither.
+// Phase A: s = the row's raw logits (q . k) in, e_j out (window rows: e_j = P_j; others relative to the
+// tile max); returns z = sum e_j.
+__device__ __forceinline__ float row_grad_a(float (&s)[64], int kind, int lo, int hi, float sc2, float lse2,
+                                            bool warp_needs_mask) {
     if (warp_needs_mask) {
         const int mlo = kind == 2 ? lo : 0, mhi = kind == 2 ? hi : 63;
 #pragma unroll
@@ -98,7 +99,7 @@ __device__ __forceinline__ RowTile row_grad(float (&s)[64], float (&dp)[64], int
     // window rows: e_j = P_j directly (base lse); other rows: base = the tile max (e_j <= 1)
     const float base = kind == 2 ? lse2 : m2;
     const float2 sc = make_float2(sc2, sc2), nb = make_float2(-base, -base);
-    float2 za[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)}, zo[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    float2 za[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
         float2 t = __ffma2_rn(make_float2(s[2 * e], s[2 * e + 1]), sc, nb);
@@ -107,19 +108,25 @@ __device__ __forceinline__ RowTile row_grad(float (&s)[64], float (&dp)[64], int
         s[2 * e] = t.x;
         s[2 * e + 1] = t.y;
         za[e & 1] = __fadd2_rn(za[e & 1], t);
-        zo[e & 1] = __ffma2_rn(t, make_float2(dp[2 * e], dp[2 * e + 1]), zo[e & 1]);
     }
-    const float z = (za[0].x + za[0].y) + (za[1].x + za[1].y);
+    return (za[0].x + za[0].y) + (za[1].x + za[1].y);
+}
+// Phase B: dp = dout . v_j in, ds_j out; s: e_j in, P_j out. beta = exp(s^_c - lse) of a selected chunk.
+// Returns ds^ of a selected chunk.
+__device__ __forceinline__ float row_grad_b(float (&s)[64], float (&dp)[64], int kind, float z, float beta,
+                                           float Dr) {
+    float2 zo[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+        zo[e & 1] = __ffma2_rn(make_float2(s[2 * e], s[2 * e + 1]), make_float2(dp[2 * e], dp[2 * e + 1]), zo[e & 1]);
     const float eo = (zo[0].x + zo[0].y) + (zo[1].x + zo[1].y);
-    RowTile rt{0.f};
-    float f = 0.f, delta = 0.f;
+    float f = 0.f, delta = 0.f, dshat = 0.f;
     if (kind == 1) {
-        const float beta = ex2_approx(sh2 - lse2);
         const float iz = 1.f / z;
         const float doo = eo * iz;
         f = beta * iz;
         delta = doo;
-        rt.dshat = beta * (doo - Dr);
+        dshat = beta * (doo - Dr);
     } else if (kind == 2) {
         f = 1.f;
         delta = Dr;
@@ -134,7 +141,7 @@ __device__ __forceinline__ RowTile row_grad(float (&s)[64], float (&dp)[64], int
         dp[2 * e] = g.x;
         dp[2 * e + 1] = g.y;
     }
-    return rt;
+    return dshat;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -153,7 +160,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap domap,
                  const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap, Dims D,
                  const int *__restrict__ ws_idx, const float *__restrict__ ws_shat, const float *__restrict__ lse,
-                 const float *__restrict__ Dbuf, __nv_bfloat16 *__restrict__ dS, int ncp, __nv_bfloat16 *__restrict__ dq) {
+                 const float *__restrict__ Dbuf, __nv_bfloat16 *__restrict__ dS, float *__restrict__ betas, int ncp,
+                 __nv_bfloat16 *__restrict__ dq) {
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) BqBars bar;
     __shared__ uint32_t s_tmem;
@@ -337,6 +345,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
             for (int t = 0; t < K; ++t)
                 if (lc[qi][t] >= 0) u = t;
         __nv_bfloat16 *dS_row = dS + row * ncp;
+        float *beta_row = betas + row * ncp;
         for (int n = grp; n < ntiles; n += 2) {
             const int bb = n & 1;
             const int c = list[n];
@@ -361,12 +370,19 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
                 float s[64], dp[64];
                 tmem_ld32(lane_base + bb * 128, *reinterpret_cast<float(*)[32]>(&s[0]));
                 tmem_ld32(lane_base + bb * 128 + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+                tmem_wait_ld();
+                // dP is loaded during the exponentials of S
                 tmem_ld32(lane_base + bb * 128 + 64, *reinterpret_cast<float(*)[32]>(&dp[0]));
                 tmem_ld32(lane_base + bb * 128 + 96, *reinterpret_cast<float(*)[32]>(&dp[32]));
-                tmem_wait_ld();
                 const bool mask = __any_sync(0xffffffffu, kind == 2 && (lo > 0 || hi < S - 1));
-                const RowTile rt = row_grad(s, dp, kind, lo, hi, sc2, lse2, sh2, Dr, mask);
-                if (kind == 1) dS_row[c] = __float2bfloat16_rn(rt.dshat);
+                const float z = row_grad_a(s, kind, lo, hi, sc2, lse2, mask);
+                tmem_wait_ld();
+                const float beta = kind == 1 ? ex2_approx(sh2 - lse2) : 0.f;
+                const float dshat = row_grad_b(s, dp, kind, z, beta, Dr);
+                if (kind == 1) {
+                    dS_row[c] = __float2bfloat16_rn(dshat);
+                    beta_row[c] = beta;  // for the KV-major kernel
+                }
 #pragma unroll
                 for (int e = 0; e < 32; ++e) pk[e] = pack_bf16(dp[2 * e], dp[2 * e + 1]);
             } else {
@@ -429,10 +445,14 @@ bwd_dqhat_kernel(Dims D, const int *__restrict__ ws_idx, const __nv_bfloat16 *__
         const int *irow = ws_idx + (((size_t)b * D.Hkv + g) * D.T + i) * K;
         const __nv_bfloat16 *drow = dS + (bh * D.T + i) * ncp;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        // lane t < K fetches slot t's id and its ds^ at once (one round trip each for the whole row),
+        // then the warp walks the slots with the values broadcast from their lanes
+        const int cl = lane < K ? irow[lane] : -1;
+        const float wl = cl >= 0 ? __bfloat162float(drow[cl]) : 0.f;
         for (int t = 0; t < K; ++t) {
-            const int c = irow[t];
+            const int c = __shfl_sync(0xffffffffu, cl, t);
             if (c < 0) break;
-            const float w = __bfloat162float(drow[c]);
+            const float w = __shfl_sync(0xffffffffu, wl, t);
             const uint2 raw = *reinterpret_cast<const uint2 *>(ks + c * 128 + 4 * lane);
             const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
             const float2 bq = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
@@ -450,7 +470,7 @@ bwd_dqhat_kernel(Dims D, const int *__restrict__ ws_idx, const __nv_bfloat16 *__
 
 // ------------------------------------------------------------------------------------------ dksum
 
-// Partial sums over one quarter of the rows of dk'[c][t] = sum_i ds^[i][c] q^[i][t] and db'[c] =
+// Partial sums over one of kDkSplit row ranges of dk'[c][t] = sum_i ds^[i][c] q^[i][t] and db'[c] =
 // sum_i ds^[i][c] for 64 chunks x 128 columns of one (b, h): four warps, 16 chunks each, mma.sync with
 // the dense ds^ matrix read transposed (A) and q^ read transposed (B); db' comes from a product with a
 // column of ones. ds^ rows have stride ncp (columns Nc..ncp-1 are zero). Partials:
@@ -628,7 +648,7 @@ struct KvBars {
 __global__ void __launch_bounds__(kTcThreads, 1)
 bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap domap,
                    const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap, Dims D,
-                   const int *__restrict__ ws_idx, const float *__restrict__ ws_shat, const float *__restrict__ lse,
+                   const float *__restrict__ betas, int ncp, const float *__restrict__ lse,
                    const float *__restrict__ Dbuf, const float *__restrict__ dk_extra, __nv_bfloat16 *__restrict__ dk,
                    __nv_bfloat16 *__restrict__ dv) {
     extern __shared__ unsigned char smem_raw[];
@@ -637,7 +657,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = D.G, QT = 128 / G;
     const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-    const int S = D.S, K = D.topk;
+    const int S = D.S;
     unsigned char *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     unsigned char *Kc = base, *Vc = base + kKvTile;
     unsigned char *QD = base + 2 * kKvTile;       // 2 stages x (Q tile, dO tile)
@@ -755,25 +775,31 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         const int qi = r / G, hh = r % G;
         const float sc2 = D.tau * kLog2e;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16);
+        // (beta of this chunk, lse in log2 units, D) of the row in query tile m: three independent loads,
+        // fetched one iteration ahead (beta = 0 where the row did not select the chunk)
+        auto fetch = [&](int m, float &beta, float &lse2, float &Dr) {
+            const int i = (qt0 + m) * QT + qi;
+            beta = 0.f;
+            lse2 = 0.f;
+            Dr = 0.f;
+            if (m < nq && i < D.T) {
+                const size_t row = ((size_t)b * D.Hq + g * G + hh) * D.T + i;
+                if (c < D.Nc) beta = betas[row * ncp + c];
+                lse2 = lse[row] * kLog2e;
+                Dr = Dbuf[row];
+            }
+        };
+        float nbeta, nlse2, nDr;
+        fetch(grp, nbeta, nlse2, nDr);
         for (int m = grp; m < nq; m += 2) {
             const int bb = m & 1;
+            const float beta = nbeta, lse2 = nlse2, Dr = nDr;
+            fetch(m + 2, nbeta, nlse2, nDr);
             const int i = (qt0 + m) * QT + qi;
             const bool valid = i < D.T;
             const int pos = D.q_pos0 + i;
             const int lpos = valid ? window_left(pos, D.W, S) : 0;
-            const size_t row = ((size_t)b * D.Hq + g * G + hh) * D.T + (valid ? i : 0);
-            bool sel = false;
-            float sh2 = 0.f;
-            if (valid && c < lpos / S) {
-                const int *irow = ws_idx + (bg * D.T + i) * K;
-                for (int t = 0; t < K; ++t) {
-                    const int cc = irow[t];
-                    if (cc == c) {
-                        sel = true;
-                        sh2 = ws_shat[row * K + t] * kLog2e;
-                    }
-                }
-            }
+            const bool sel = valid && beta > 0.f;
             int lo = 0, hi = S - 1;
             if (valid && !sel) {
                 lo = max(lpos - j0, 0);
@@ -781,8 +807,6 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
             }
             const bool win = valid && !sel && lo <= hi;
             const int kind = sel ? 1 : (win ? 2 : 0);
-            const float lse2 = valid ? lse[row] * kLog2e : 0.f;
-            const float Dr = valid ? Dbuf[row] : 0.f;
             if (__any_sync(0xffffffffu, !mbar_wait_bounded(&bar.s_full[bb], (m >> 1) & 1))) {
                 ok = false;
                 break;
@@ -793,11 +817,14 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
                 float s[64], dp[64];
                 tmem_ld32(lane_base + bb * 128, *reinterpret_cast<float(*)[32]>(&s[0]));
                 tmem_ld32(lane_base + bb * 128 + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+                tmem_wait_ld();
+                // dP is loaded during the exponentials of S
                 tmem_ld32(lane_base + bb * 128 + 64, *reinterpret_cast<float(*)[32]>(&dp[0]));
                 tmem_ld32(lane_base + bb * 128 + 96, *reinterpret_cast<float(*)[32]>(&dp[32]));
-                tmem_wait_ld();
                 const bool mask = __any_sync(0xffffffffu, kind == 2 && (lo > 0 || hi < S - 1));
-                row_grad(s, dp, kind, lo, hi, sc2, lse2, sh2, Dr, mask);
+                const float z = row_grad_a(s, kind, lo, hi, sc2, lse2, mask);
+                tmem_wait_ld();
+                row_grad_b(s, dp, kind, z, beta, Dr);
 #pragma unroll
                 for (int x = 0; x < 8; ++x) {
                     pw[x] = make_uint4(pack_bf16(s[8 * x], s[8 * x + 1]), pack_bf16(s[8 * x + 2], s[8 * x + 3]),
@@ -864,7 +891,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
 int ds_stride(const Dims &D) { return (std::max(D.Nc, 1) + 7) & ~7; }
 
 struct BwdLayout {
-    size_t idx, shat, dbuf, ds, part, dkx, total;
+    size_t idx, shat, dbuf, ds, beta, part, dkx, total;
 };
 
 BwdLayout bwd_layout(const Dims &D) {
@@ -879,6 +906,7 @@ BwdLayout bwd_layout(const Dims &D) {
     L.shat = take((size_t)D.B * D.Hq * D.T * D.topk * sizeof(float));
     L.dbuf = take((size_t)D.B * D.Hq * D.T * sizeof(float));
     L.ds = take((size_t)D.B * D.Hq * D.T * ds_stride(D) * sizeof(__nv_bfloat16));
+    L.beta = take((size_t)D.B * D.Hq * D.T * ds_stride(D) * sizeof(float));
     L.part = take((size_t)D.B * D.Hq * kDkSplit * std::max(D.Nc, 1) * kPartStride * sizeof(float));
     L.dkx = take((size_t)D.B * D.Hkv * D.L * 128 * sizeof(float));
     L.total = off;
@@ -915,6 +943,7 @@ cudaError_t launch_attn_bwd_tc(const Dims &D, const void *q, const void *k, cons
     float *ws_shat = (float *)(w + L.shat);
     float *Dbuf = (float *)(w + L.dbuf);
     __nv_bfloat16 *dS = (__nv_bfloat16 *)(w + L.ds);
+    float *betas = (float *)(w + L.beta);
     float *part = (float *)(w + L.part);
     float *dkx = (float *)(w + L.dkx);
     cudaError_t e = launch_gather_shat_tc(D, q_hat, k_sum, b_sum, idx, ws_idx, ws_shat, stream);
@@ -924,6 +953,8 @@ cudaError_t launch_attn_bwd_tc(const Dims &D, const void *q, const void *k, cons
         (const __nv_bfloat16 *)out, (const __nv_bfloat16 *)dout, Dbuf, rows);
     const int ncp = ds_stride(D);
     e = cudaMemsetAsync(dS, 0, (size_t)rows * ncp * sizeof(__nv_bfloat16), stream);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(betas, 0, (size_t)rows * ncp * sizeof(float), stream);
     if (e != cudaSuccess) return e;
     const int QT = 128 / D.G;
     CUtensorMap qmap, domap, kmap, vmap;
@@ -937,7 +968,7 @@ cudaError_t launch_attn_bwd_tc(const Dims &D, const void *q, const void *k, cons
         const size_t smem = 1024 + 2 * kRowTile + 2 * kBqStages * kKvTile;
         cudaFuncSetAttribute(bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         bwd_dq_tc_kernel<<<dim3((D.T + QT - 1) / QT, D.Hkv, D.B), kTcThreads, smem, stream>>>(
-            qmap, domap, kmap, vmap, D, ws_idx, ws_shat, lse, Dbuf, dS, ncp, (__nv_bfloat16 *)dq);
+            qmap, domap, kmap, vmap, D, ws_idx, ws_shat, lse, Dbuf, dS, betas, ncp, (__nv_bfloat16 *)dq);
     }
     if (D.Nc > 0) {
         bwd_dqhat_kernel<<<dim3((D.T + 255) / 256, D.Hq, D.B), 256, 0, stream>>>(
@@ -955,7 +986,7 @@ cudaError_t launch_attn_bwd_tc(const Dims &D, const void *q, const void *k, cons
         const size_t smem = 1024 + 2 * kKvTile + 4 * kRowTile + 2 * kKvTile;
         cudaFuncSetAttribute(bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         bwd_dkdv_tc_kernel<<<dim3((D.L + D.S - 1) / D.S, D.Hkv, D.B), kTcThreads, smem, stream>>>(
-            qmap, domap, kmap, vmap, D, ws_idx, ws_shat, lse, Dbuf, dkx, (__nv_bfloat16 *)dk, (__nv_bfloat16 *)dv);
+            qmap, domap, kmap, vmap, D, betas, ncp, lse, Dbuf, dkx, (__nv_bfloat16 *)dk, (__nv_bfloat16 *)dv);
     }
     return cudaGetLastError();
 }
