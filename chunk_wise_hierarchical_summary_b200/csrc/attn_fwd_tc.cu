@@ -49,9 +49,10 @@ struct Bars {
     // p_full is per S/P buffer: a row warp may run one tile ahead (its next S is ready before every warp
     // has written this tile's P), so one shared barrier would let an early arrival complete a phase.
     // o_final completes once, after the last value product: the row warps' epilogue cannot wait on a
-    // pv_done parity, because a warp that skipped per-tile waits may see pv_done two phases behind.
-    uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages], s_full[2], p_full[2],
-        pv_done, o_final;
+    // pv_done parity, because a warp that skipped per-tile waits may see pv_done several phases behind.
+    // With two stages and two S buffers, stage n % 2 and buffer n & 1 coincide: s_full[b] also frees K stage
+    // b (the QK product read it) and pv_done[b] frees V stage b, so each MMA group needs one commit.
+    uint64_t q_full, k_full[kStages], v_full[kStages], s_full[2], p_full[2], pv_done[2], o_final;
 };
 
 __global__ void __launch_bounds__(kThreads, 2)
@@ -86,15 +87,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         mbar_init(&bar.q_full, 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&bar.k_full[s], 1);
-            mbar_init(&bar.k_empty[s], 1);
             mbar_init(&bar.v_full[s], 1);
-            mbar_init(&bar.v_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bar.s_full[s], 1);
             mbar_init(&bar.p_full[s], 128);
+            mbar_init(&bar.pv_done[s], 1);
         }
-        mbar_init(&bar.pv_done, 1);
         mbar_init(&bar.o_final, 1);
         fence_mbar_init();
     }
@@ -159,7 +158,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             const int kvrow0 = (b * D.Hkv + g) * D.L;
             auto load_k = [&](int n) {
                 const int st = n % kStages;
-                if (n >= kStages && !mbar_wait_bounded(&bar.k_empty[st], ((n / kStages) - 1) & 1)) return false;
+                if (n >= kStages && !mbar_wait_bounded(&bar.s_full[st], ((n / kStages) - 1) & 1)) return false;
                 unsigned char *Kt = Ks + st * kTileBytes;
                 const int y = kvrow0 + list[n] * S;
                 mbar_arrive_expect_tx(&bar.k_full[st], kTileBytes);
@@ -169,7 +168,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             };
             auto load_v = [&](int n) {
                 const int st = n % kStages;
-                if (n >= kStages && !mbar_wait_bounded(&bar.v_empty[st], ((n / kStages) - 1) & 1)) return false;
+                if (n >= kStages && !mbar_wait_bounded(&bar.pv_done[st], ((n / kStages) - 1) & 1)) return false;
                 unsigned char *Vt = Vs + st * kTileBytes;
                 const int y = kvrow0 + list[n] * S;
                 mbar_arrive_expect_tx(&bar.v_full[st], kTileBytes);
@@ -200,15 +199,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                 for (int ks = 0; ks < 4; ++ks)
                     umma_bf16_tmem_a(tmem + 128, pa + ks * 8, sdesc_sw128(va + ks * 2048, 8192, 1024), idesc_pv,
                                      (n > 0 || ks > 0) ? 1u : 0u);
-                umma_commit(&bar.pv_done);
-                umma_commit(&bar.v_empty[st]);
+                umma_commit(&bar.pv_done[n & 1]);
                 return true;
             };
             for (int n = 0; n < ntiles && ok; ++n) {
                 const int st = n % kStages, sb = n & 1;
                 if (!mbar_wait_bounded(&bar.k_full[st], (n / kStages) & 1)) { ok = false; break; }
                 // S/P buffer sb held P(n-2): reuse it only after PV(n-2) has completed
-                if (n >= 2 && !mbar_wait_bounded(&bar.pv_done, (n - 2) & 1)) { ok = false; break; }
+                if (n >= 2 && !mbar_wait_bounded(&bar.pv_done[sb], ((n - 2) >> 1) & 1)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t ka = smem_u32(Ks + st * kTileBytes);
 #pragma unroll
@@ -219,7 +217,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                               idesc_qk, ks > 0 ? 1u : 0u);
                 }
                 umma_commit(&bar.s_full[sb]);
-                umma_commit(&bar.k_empty[st]);
                 if (n >= 1) {
                     if (!mbar_wait_bounded(&bar.p_full[(n - 1) & 1], ((n - 1) >> 1) & 1)) { ok = false; break; }
                     tc_fence_after();
@@ -343,7 +340,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             // O rescale (rare; warp-collective TMEM access) once PV(n-1) has completed
             const unsigned need = __ballot_sync(0xffffffffu, factor != 1.f && n >= 1);
             if (need) {
-                if (__any_sync(0xffffffffu, !mbar_wait_bounded(&bar.pv_done, (n - 1) & 1))) {
+                if (__any_sync(0xffffffffu, !mbar_wait_bounded(&bar.pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1))) {
                     ok = false;
                     break;
                 }
