@@ -222,16 +222,21 @@ def prefill_work(w: W.Workload):
 
 
 def decode_bytes(w: W.Workload):
-    """Bytes one decode step must touch: every candidate summary (k' in the input dtype + fp32 b'),
-    the selected chunks' K and V, the window's K and V, q, q^ and the output."""
+    """Bytes one decode step must touch for its M = w.T queries at the end of the cache: every candidate
+    summary once (k' in the input dtype + fp32 b'; the last query's candidates, the most), and per query
+    its selected chunks' K and V, its window's K and V, and q, q^ and the output."""
     el = 2 if w.dtype == "bf16" else 4
-    p = w.L - 1
-    l = window_left(p, w.W, w.S)
-    n = l // w.S
-    summ = w.B * w.Hq * n * (w.d * el + 4)
-    chunks = w.B * w.Hkv * min(w.topk, n) * w.S * w.d * el * 2
-    win = w.B * w.Hkv * (p - l + 1) * w.d * el * 2
-    io = w.B * w.Hq * w.d * el * 3 + w.B * w.Hq * 4
+    M = w.T
+    p_last = w.L - 1
+    n_last = window_left(p_last, w.W, w.S) // w.S
+    summ = w.B * w.Hq * n_last * (w.d * el + 4)
+    chunks = win = 0
+    for m in range(M):
+        p = w.L - M + m
+        l = window_left(p, w.W, w.S)
+        chunks += w.B * w.Hkv * min(w.topk, l // w.S) * w.S * w.d * el * 2
+        win += w.B * w.Hkv * (p - l + 1) * w.d * el * 2
+    io = w.B * w.Hq * M * (w.d * el * 3 + 4)
     return {"total": summ + chunks + win + io, "summaries": summ, "chunks": chunks, "window": win, "io": io}
 
 
@@ -334,9 +339,10 @@ def bench_decode(args, dist, dev, H, peaks, w: W.Workload, steps: int):
     el = 2 if w.dtype == "bf16" else 4
     summ_bytes = (w.B * w.Hkv * w.Nc * w.S * w.d * el + 2 * w.B * w.Hq * w.Nc * w.d * el + 4 * w.B * w.Hq * w.Nc)
     out = torch.empty_like(x["q"])
-    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
-    idx = torch.empty((w.B, w.Hkv, w.topk), dtype=torch.int32, device=dev)
-    p = H.make_params(w.B, 1, w.L, w.Hq, w.Hkv, w.d, w.S, w.topk, w.W, w.L - 1)
+    M = w.T
+    lse = torch.empty((w.B, w.Hq) if M == 1 else (w.B, w.Hq, M), dtype=torch.float32, device=dev)
+    idx = torch.empty((w.B, w.Hkv, w.topk) if M == 1 else (w.B, w.Hkv, M, w.topk), dtype=torch.int32, device=dev)
+    p = H.make_params(w.B, M, w.L, w.Hq, w.Hkv, w.d, w.S, w.topk, w.W, w.L - M)
     ws = torch.empty(H.workspace_size(p, H.OP_DECODE), dtype=torch.uint8, device=dev)
 
     def one():
@@ -360,11 +366,12 @@ def bench_decode(args, dist, dev, H, peaks, w: W.Workload, steps: int):
         graph.replay()
         mark()
 
-    _, total_ms, clocks = timed_steps(1, run, max(1, args.warmup // 3), None, dist,
+    _, total_ms, clocks = timed_steps(1, run, max(3, args.warmup // 3), None, dist,
                                       ClockSampler(physical_gpu_index(dist.local_rank)))
     needles_found = 0
     for b in range(w.B):
-        needles_found += len(set(x["needle_chunks"][b].tolist()) & set(idx[b, 0].tolist()))
+        first = idx[b, 0] if w.T == 1 else idx[b, 0, 0]  # the needle keys follow the first query's q^
+        needles_found += len(set(x["needle_chunks"][b].tolist()) & set(first.tolist()))
     ms_step = dist.max(total_ms / steps)  # per-sequence-batch latency: the slowest rank's
     nbytes = decode_bytes(w)
     gbs = nbytes["total"] / (ms_step / 1e3) / 1e9
@@ -372,7 +379,8 @@ def bench_decode(args, dist, dev, H, peaks, w: W.Workload, steps: int):
     summ = {"ms": summ_ms, "bytes": summ_bytes, "achieved_gbs": summ_bytes / (summ_ms / 1e3) / 1e9,
             "peak_gbs": peaks["hbm_gbs"], "frac": summ_bytes / (summ_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
             "note": "hils_chunk_summary over the whole cache: K and landmark queries read, k' and b' written"}
-    return {"workload": w.name, "us_per_token": ms_step * 1e3, "us_per_step_per_seq": ms_step * 1e3 / w.B,
+    return {"workload": w.name, "query_tokens_per_step": M, "us_per_step": ms_step * 1e3,
+            "us_per_token": ms_step * 1e3 / M, "us_per_step_per_seq": ms_step * 1e3 / w.B,
             "summaries": summ,
             "steps": steps, "bytes_per_step": nbytes,
             "roofline": {"bound": "hbm", "kernel": "hils_decode (whole step: score, select, attend, combine)",
@@ -578,6 +586,10 @@ def main():
                 extra["decode_sweep"].append({"L": L, "us_per_token": r["us_per_token"],
                                               "bytes_per_step": r["bytes_per_step"]["total"],
                                               "hbm_frac": r["roofline"]["frac"], "needle_recall": r["needle_recall"]})
+            # multi-token decode (M = 4 query tokens per sequence and step, e.g. speculative verification)
+            wm = W.DECODE_BF16.with_(name="decode_m4_bf16_B8_L524288_Hq32_Hkv8_d128_S64_k32_W512", T=4,
+                                     q_pos0=W.DECODE_BF16.L - 4)
+            extra["decode_multi"] = bench_decode(args, dist, dev, H, peaks, wm, 64)
             extra["train"] = bench_train(args, dist, dev, H, peaks)
         cpu = None
         if dist.world == 1:

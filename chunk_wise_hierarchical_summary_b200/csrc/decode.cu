@@ -17,6 +17,8 @@
 //              chunk or a window tile) per CTA, K and V staged by bulk copies, all G heads, a partial
 //              (max, sum, acc[d]) of the online softmax over adjusted logits (a chunk token carries
 //              s_j - L_c + s^_c); the last CTA of each (b, KV group) merges the partials into out, lse.
+#include <algorithm>
+
 #include "internal.h"
 #include "tma.cuh"
 
@@ -27,6 +29,10 @@ cudaError_t launch_decode_attn_mma(const Dims &D, int n, int ntiles, const void 
                                    const void *v_cache, const float *scores, const int *sel, float *partial,
                                    unsigned int *counters, void *out, float *lse, cudaStream_t stream);
 unsigned int decode_attn_mma_error_flags(bool clear);
+bool decode_score_mma_supported(const Dims &D, int dtype, const void *q_hat, const void *k_sum);
+cudaError_t launch_decode_score_mma(const Dims &D, int n, int nslices, const void *q_hat, const void *k_sum,
+                                    const float *b_sum, float *scores, float *part, cudaStream_t stream);
+unsigned int decode_score_mma_error_flags(bool clear);
 
 namespace {
 
@@ -53,14 +59,21 @@ constexpr int kSliceElems = 16384;  // summary elements per scored slice
 constexpr int kScorePartsPerSliceHost = 4;  // partials per slice (one per consumer warp of a slot)
 
 DecodePlan make_plan(const Dims &D) {
+    // M = D.T query tokens at positions q_pos0 .. q_pos0 + M - 1 = L - 1 (M = 1: plain decode). The score
+    // rows span the last query's candidates (the most); every other query masks to its own.
     DecodePlan P{};
-    const int pos = D.L - 1;
+    const int M = D.T;
+    const int pos = D.q_pos0 + M - 1;
     const int l = window_left(pos, D.W, D.S);
     P.n = l / D.S;
     const int bg = D.B * D.Hkv;
     P.per = kSliceElems / D.d;  // 128 rows at d 128
     P.nslices = P.n > 0 ? (P.n + P.per - 1) / P.per : 1;
-    P.wtiles = (pos - l + 1 + D.S - 1) / D.S;
+    P.wtiles = 0;
+    for (int m = 0; m < M; ++m) {
+        const int pm = D.q_pos0 + m, lm = window_left(pm, D.W, D.S);
+        P.wtiles = std::max(P.wtiles, (pm - lm + 1 + D.S - 1) / D.S);
+    }
     P.ntiles = D.topk + P.wtiles;
     P.nparts = P.n > 0 ? (P.n + kSelPart - 1) / kSelPart : 1;
     size_t off = 0;
@@ -69,13 +82,13 @@ DecodePlan make_plan(const Dims &D) {
         off += (bytes + 255) & ~(size_t)255;
         return at;
     };
-    P.off_scores = take((size_t)D.B * D.Hq * (P.n > 0 ? P.n : 1) * sizeof(float));
-    P.off_part = take((size_t)D.B * D.Hq * P.nslices * kScorePartsPerSliceHost * 2 * sizeof(float));
-    P.off_list = take((size_t)bg * P.nparts * D.topk * sizeof(uint64_t));
-    P.off_sel = take((size_t)bg * D.topk * sizeof(int));
-    P.off_attn = take((size_t)D.B * D.Hq * P.ntiles * (D.d + 4) * sizeof(float));  // either attention form
-    P.off_count = take((size_t)bg * sizeof(unsigned int));
-    P.off_selcount = take((size_t)bg * sizeof(unsigned int));
+    P.off_scores = take((size_t)D.B * D.Hq * M * (P.n > 0 ? P.n : 1) * sizeof(float));
+    P.off_part = take((size_t)D.B * D.Hq * M * P.nslices * kScorePartsPerSliceHost * 2 * sizeof(float));
+    P.off_list = take((size_t)bg * M * P.nparts * D.topk * sizeof(uint64_t));
+    P.off_sel = take((size_t)bg * M * D.topk * sizeof(int));
+    P.off_attn = take((size_t)D.B * D.Hq * M * P.ntiles * (D.d + 4) * sizeof(float));  // either attention form
+    P.off_count = take((size_t)bg * M * sizeof(unsigned int));
+    P.off_selcount = take((size_t)bg * M * sizeof(unsigned int));
     P.total = off;
     return P;
 }
@@ -497,8 +510,8 @@ __device__ __forceinline__ uint64_t warp_merge_lowest32(uint64_t a, uint64_t b) 
 // candidates, merged in registers batch by batch, and the CTA reduces the warps' lists. Returns the 32
 // smallest keys, ascending, to warp 0 (one per lane).
 template <int GM>
-__device__ __noinline__ uint64_t select_tied_fallback(const float *__restrict__ sc0, int G, int n, int rounds,
-                                                      const float (&L)[8], uint64_t *keys) {
+__device__ __noinline__ uint64_t select_tied_fallback(const float *__restrict__ sc0, size_t hs, int G, int n,
+                                                      int rounds, const float (&L)[8], uint64_t *keys) {
     constexpr int kPer = 64 / GM, kRound = 512 * kPer;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     uint64_t best = ~0ull;
@@ -509,7 +522,7 @@ __device__ __noinline__ uint64_t select_tied_fallback(const float *__restrict__ 
             for (int i = 0; i < 8; ++i) {
                 const int c = r * kRound + warp * (32 * kPer) + (h * 8 + i) * 32 + lane;
                 float gv = -INFINITY;
-                for (int hh = 0; hh < G; ++hh) gv = fmaxf(gv, (c < n ? sc0[(size_t)hh * n + c] : -INFINITY) - L[hh]);
+                for (int hh = 0; hh < G; ++hh) gv = fmaxf(gv, (c < n ? sc0[hh * hs + c] : -INFINITY) - L[hh]);
                 kv[i] = (c < n) ? desc_value_key(gv, (uint32_t)c) : ~0ull;
             }
             warp_bitonic_sort<8>(kv);
@@ -552,12 +565,15 @@ decode_select_warp_kernel(Dims D, DecodePlan P, const float *__restrict__ scores
     __shared__ __align__(8) uint64_t surv[kSelWCap];
     __shared__ uint64_t s_bound;
     __shared__ int s_count;
-    const int g = blockIdx.x, b = blockIdx.y;
-    const int G = D.G, K = D.topk, n = P.n;
-    const size_t bg = (size_t)b * D.Hkv + g;
+    // grid (Hkv, B * M): query m of sequence b; its candidates are the chunks before its window
+    const int g = blockIdx.x, M = D.T, b = blockIdx.y / M, m = blockIdx.y % M;
+    const int G = D.G, K = D.topk;
+    const int n = window_left(D.q_pos0 + m, D.W, D.S) / D.S;
+    const size_t bgm = ((size_t)b * D.Hkv + g) * M + m;
+    const size_t hs = (size_t)M * P.n;  // stride between the group's heads in the score rows
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = kSelWThreads / 32;
-    int *out = sel + bg * K;
-    int *out2 = idx_out ? idx_out + bg * K : nullptr;
+    int *out = sel + bgm * K;
+    int *out2 = idx_out ? idx_out + bgm * K : nullptr;
     if (n == 0) {
         for (int t = tid; t < K; t += blockDim.x) {
             out[t] = -1;
@@ -565,7 +581,7 @@ decode_select_warp_kernel(Dims D, DecodePlan P, const float *__restrict__ scores
         }
         return;
     }
-    const float *sc0 = scores + ((size_t)b * D.Hq + g * G) * n;
+    const float *sc0 = scores + (((size_t)b * D.Hq + g * G) * M + m) * P.n;
     constexpr int kSelWPer = 64 / GM;                     // candidates per thread per round
     constexpr int kSelWRound = kSelWThreads * kSelWPer;
     const int rounds = (n + kSelWRound - 1) / kSelWRound;
@@ -578,7 +594,7 @@ decode_select_warp_kernel(Dims D, DecodePlan P, const float *__restrict__ scores
 #pragma unroll
             for (int i = 0; i < kSelWPer; ++i) {
                 const int c = cand(r, i);
-                raw[hh][i] = (hh < G && c < n) ? sc0[(size_t)hh * n + c] : -INFINITY;
+                raw[hh][i] = (hh < G && c < n) ? sc0[hh * hs + c] : -INFINITY;
             }
     };
     load_round(0);  // in flight during the LSE fold
@@ -586,7 +602,7 @@ decode_select_warp_kernel(Dims D, DecodePlan P, const float *__restrict__ scores
     if (warp < G) {
         const int hh = warp;
         const int np = P.nslices * kScorePartsPerSliceHost;
-        const float2 *ph = reinterpret_cast<const float2 *>(part + ((size_t)b * D.Hq + g * G + hh) * np * 2);
+        const float2 *ph = reinterpret_cast<const float2 *>(part + (((size_t)b * D.Hq + g * G + hh) * M + m) * np * 2);
         float M = -INFINITY, Z = 0.f;
         for (int s0 = 0; s0 < np; s0 += 32 * 8) {
             float2 v[8];
@@ -684,7 +700,7 @@ decode_select_warp_kernel(Dims D, DecodePlan P, const float *__restrict__ scores
             top = warp_first32<4>(kv);
         }
     } else {
-        top = select_tied_fallback<GM>(sc0, G, n, rounds, L, keys);
+        top = select_tied_fallback<GM>(sc0, hs, G, n, rounds, L, keys);
     }
     if (warp == 0) {
         // the selected ids (first min(K, n) keys), written ascending, -1 padded
@@ -912,7 +928,10 @@ cudaError_t launch_t(const Dims &D, const void *q, const void *q_hat, const void
     // Both counter arrays (attention, selection) are adjacent: clear them in one call.
     cudaError_t e = cudaMemsetAsync(counters, 0, P.total - P.off_count, stream);
     if (e != cudaSuccess) return e;
-    if (P.n > 0) {
+    if (P.n > 0 && D.T > 1) {
+        cudaError_t es = launch_decode_score_mma(D, P.n, P.nslices, q_hat, k_sum, b_sum, scores, part, stream);
+        if (es != cudaSuccess) return es;
+    } else if (P.n > 0) {
         using C = ScoreCfg<T>;
         static_assert(C::kWarpsPerSlot == kScorePartsPerSliceHost, "one partial per consumer warp of a slot");
         const size_t smem1 = (size_t)C::kStages * P.per * D.d * sizeof(T) +
@@ -927,9 +946,11 @@ cudaError_t launch_t(const Dims &D, const void *q, const void *q_hat, const void
     }
     unsigned int *selcount = (unsigned int *)(w + P.off_selcount);
     if (D.topk <= 32 && D.G <= 4)
-        decode_select_warp_kernel<4><<<dim3(D.Hkv, D.B), kSelWThreads, 0, stream>>>(D, P, scores, part, sel, idx_out);
+        decode_select_warp_kernel<4><<<dim3(D.Hkv, D.B * D.T), kSelWThreads, 0, stream>>>(D, P, scores, part, sel,
+                                                                                          idx_out);
     else if (D.topk <= 32 && D.G <= 8)
-        decode_select_warp_kernel<8><<<dim3(D.Hkv, D.B), kSelWThreads, 0, stream>>>(D, P, scores, part, sel, idx_out);
+        decode_select_warp_kernel<8><<<dim3(D.Hkv, D.B * D.T), kSelWThreads, 0, stream>>>(D, P, scores, part, sel,
+                                                                                          idx_out);
     else
         decode_select_kernel<<<dim3(P.nparts, D.Hkv, D.B), kSelThreads, 0, stream>>>(D, P, scores, part, lists,
                                                                                      selcount, sel, idx_out);
@@ -960,8 +981,18 @@ bool decode_supported(const Dims &D) {
            smem3 <= 200 * 1024;
 }
 
+// M > 1 query tokens run on the bf16 d 128 S 64 kernels only (streamed scores, single-CTA selection,
+// split-K attention); the general kernels are single-token.
+bool decode_multi_supported(const Dims &D, int dtype, const void *q, const void *q_hat, const void *k,
+                            const void *v, const void *k_sum) {
+    if (D.T == 1) return true;
+    const DecodePlan P = make_plan(D);
+    return D.T <= 8 && D.topk <= 32 && D.G <= 8 && decode_score_mma_supported(D, dtype, q_hat, k_sum) &&
+           decode_attn_mma_supported(D, dtype, q, k, v, P.ntiles);
+}
+
 unsigned int decode_error_flags(bool clear) {
-    unsigned int v = decode_attn_mma_error_flags(clear);
+    unsigned int v = decode_attn_mma_error_flags(clear) | decode_score_mma_error_flags(clear);
     unsigned int mine = 0;
     cudaMemcpyFromSymbol(&mine, g_decode_errors, sizeof(mine));
     v |= mine;

@@ -2,8 +2,9 @@
 // over its selected chunks and its window, fused by Eq. 10 ("Hierarchical Sparse Attention Done Right",
 // Sec. 3 RQ2, Eq. 10; Sec. 4 "GQA": the group's heads share every gathered tile).
 //
-// grid (nsplit, Hkv, B): the tiles of one (b, KV group) - its selected chunks, then its window tiles -
-// are dealt round-robin to nsplit CTAs. Per CTA:
+// grid (nsplit, Hkv, B * M) for M = T query tokens per sequence (M > 1: multi-token decode): the tiles of
+// one (b, KV group, query) - its selected chunks, then its window tiles - are dealt round-robin to
+// nsplit CTAs. Per CTA:
 //   warp 4     producer: K and V tiles (TMA, 128-byte swizzle) into a kStages-deep ring.
 //   warps 0-3  per tile, on the warp-level tensor-core instruction (mma.sync m16n8k16, bf16 in, fp32
 //              accumulate) with the group's heads as the 8-wide N side:
@@ -59,11 +60,14 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     __shared__ Tile tiles[kMaxTiles];
     __shared__ int s_nt, s_last;
     unsigned char *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-    const int split = blockIdx.x, nsplit = gridDim.x, g = blockIdx.y, b = blockIdx.z;
+    // grid z = b * M + m: query m (of M = D.T, at position q_pos0 + m) of sequence b
+    const int split = blockIdx.x, nsplit = gridDim.x, g = blockIdx.y, M = D.T;
+    const int b = blockIdx.z / M, m = blockIdx.z % M;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = D.G, S = D.S, K = D.topk;
-    const size_t bg = (size_t)b * D.Hkv + g;
-    const int pos = D.L - 1;
+    const size_t bg = (size_t)b * D.Hkv + g;  // K/V rows
+    const size_t bgm = bg * M + m;            // this query's ids and counter
+    const int pos = D.q_pos0 + m;
     const int l = window_left(pos, D.W, S);
 
     if (tid == 0) {
@@ -76,7 +80,7 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
         for (int t = split; t < ntiles && nt < kMaxTiles; t += nsplit) {
             Tile tl;
             if (t < K) {
-                const int c = sel[bg * K + t];
+                const int c = sel[bgm * K + t];
                 if (c < 0) continue;
                 tl.j0 = c * S;
                 tl.jn = S;
@@ -94,7 +98,7 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     for (int e = tid; e < G * 16; e += blockDim.x) {  // the group's query rows, 16 bytes per thread
         const int h = e >> 4, ch = e & 15;
         *reinterpret_cast<uint4 *>(qs + h * kQRowBytes + ch * 16) =
-            *reinterpret_cast<const uint4 *>(q + ((size_t)b * D.Hq + g * G + h) * 128 + ch * 8);
+            *reinterpret_cast<const uint4 *>(q + (((size_t)b * D.Hq + g * G + h) * M + m) * 128 + ch * 8);
     }
     __syncthreads();
     const int nt = s_nt;
@@ -129,15 +133,16 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
         const int mi = lane >> 3, r8 = lane & 7;
         const bool hv = g8 < G;
         const float sc2 = D.tau * kLog2e;
-        const size_t hrow0 = (size_t)b * D.Hq + g * G;
+        // query rows (b, head, m) of [B, Hq, M, ...]: head h of the group at hrow0 + h * M
+        const size_t hrow0 = ((size_t)b * D.Hq + g * G) * M + m;
         for (int i = 0; i < nt; ++i) {
             const int st = i % kStages;
             const Tile tl = tiles[i];
             // the chunk's retrieval score for this thread's two heads, fetched before the tile wait
             float sh0 = 0.f, sh1 = 0.f;
             if (tl.c >= 0) {
-                if (2 * t4 < G) sh0 = scores[(hrow0 + 2 * t4) * n + tl.c] * kLog2e;
-                if (2 * t4 + 1 < G) sh1 = scores[(hrow0 + 2 * t4 + 1) * n + tl.c] * kLog2e;
+                if (2 * t4 < G) sh0 = scores[(hrow0 + (size_t)(2 * t4) * M) * n + tl.c] * kLog2e;
+                if (2 * t4 + 1 < G) sh1 = scores[(hrow0 + (size_t)(2 * t4 + 1) * M) * n + tl.c] * kLog2e;
             }
             const bool got = mbar_wait_bounded(&full[st], (i / kStages) & 1);
             const uint32_t Kb = smem_u32(base + st * 2 * kTileBytes), Vb = Kb + kTileBytes;
@@ -246,24 +251,24 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
             for (int mt = 0; mt < 2; ++mt) {
                 const int dd = 32 * warp + 16 * mt + g8;
                 if (2 * t4 < G) {
-                    float *pp = partial + ((hrow0 + 2 * t4) * nsplit + split) * kPartStride + 4;
+                    float *pp = partial + ((hrow0 + (size_t)(2 * t4) * M) * nsplit + split) * kPartStride + 4;
                     pp[dd] = o[mt][0];
                     pp[dd + 8] = o[mt][2];
                 }
                 if (2 * t4 + 1 < G) {
-                    float *pp = partial + ((hrow0 + 2 * t4 + 1) * nsplit + split) * kPartStride + 4;
+                    float *pp = partial + ((hrow0 + (size_t)(2 * t4 + 1) * M) * nsplit + split) * kPartStride + 4;
                     pp[dd] = o[mt][1];
                     pp[dd + 8] = o[mt][3];
                 }
             }
             if (warp == 0 && g8 == 0) {
                 if (2 * t4 < G) {
-                    float *pp = partial + ((hrow0 + 2 * t4) * nsplit + split) * kPartStride;
+                    float *pp = partial + ((hrow0 + (size_t)(2 * t4) * M) * nsplit + split) * kPartStride;
                     pp[0] = M0;
                     pp[1] = l0;
                 }
                 if (2 * t4 + 1 < G) {
-                    float *pp = partial + ((hrow0 + 2 * t4 + 1) * nsplit + split) * kPartStride;
+                    float *pp = partial + ((hrow0 + (size_t)(2 * t4 + 1) * M) * nsplit + split) * kPartStride;
                     pp[0] = M1;
                     pp[1] = l1;
                 }
@@ -274,24 +279,27 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     __syncthreads();
     if (tid == 0) {
         __threadfence();
-        s_last = (atomicAdd(&counters[bg], 1u) == (unsigned)(nsplit - 1));
+        s_last = (atomicAdd(&counters[bgm], 1u) == (unsigned)(nsplit - 1));
     }
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    // merge the nsplit partials of each head: one warp per head, lane owns 4 columns
+    // merge the nsplit (<= 32) partials of each head: one warp per head. Lane s fetches split s's (M, l),
+    // the warp reduces them, then each lane accumulates its 4 columns over the splits, four loads in
+    // flight at a time.
     for (int hh = warp; hh < G; hh += blockDim.x >> 5) {
-        const size_t hr = (size_t)b * D.Hq + g * G + hh;
+        const size_t hr = ((size_t)b * D.Hq + g * G + hh) * M + m;
         const float *ph = partial + hr * nsplit * kPartStride;
-        float M = -INFINITY;
-        for (int s = 0; s < nsplit; ++s) M = fmaxf(M, __ldcg(ph + (size_t)s * kPartStride));
-        float Z = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int s = 0; s < nsplit; ++s) {
-            const float ms = __ldcg(ph + (size_t)s * kPartStride);
-            if (ms == -INFINITY) continue;  // a CTA with no tiles
-            const float r = ex2_approx(ms - M);
-            Z += __ldcg(ph + (size_t)s * kPartStride + 1) * r;
-            const float4 v4 = __ldcg(reinterpret_cast<const float4 *>(ph + (size_t)s * kPartStride + 4) + lane);
+        const float ms = lane < nsplit ? __ldcg(ph + (size_t)lane * kPartStride) : -INFINITY;
+        const float ls = lane < nsplit ? __ldcg(ph + (size_t)lane * kPartStride + 1) : 0.f;
+        const float Mx = warp_max(ms);
+        const float rs = ms == -INFINITY ? 0.f : ex2_approx(ms - Mx);  // a CTA with no tiles has weight 0
+        const float Z = warp_sum(ls * rs);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+        for (int s2 = 0; s2 < nsplit; ++s2) {
+            const float r = __shfl_sync(0xffffffffu, rs, s2);
+            const float4 v4 = __ldcg(reinterpret_cast<const float4 *>(ph + (size_t)s2 * kPartStride + 4) + lane);
             acc[0] = fmaf(v4.x, r, acc[0]);
             acc[1] = fmaf(v4.y, r, acc[1]);
             acc[2] = fmaf(v4.z, r, acc[2]);
@@ -304,7 +312,7 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
         w2.x = *reinterpret_cast<const uint32_t *>(&h01);
         w2.y = *reinterpret_cast<const uint32_t *>(&h23);
         *reinterpret_cast<uint2 *>(out + hr * 128 + lane * 4) = w2;
-        if (lane == 0) lse[hr] = (M + log2f(Z)) * (1.f / kLog2e);
+        if (lane == 0) lse[hr] = (Mx + log2f(Z)) * (1.f / kLog2e);
     }
 }
 
@@ -316,10 +324,11 @@ bool decode_attn_mma_supported(const Dims &D, int dtype, const void *q, const vo
            al16(q) && al16(k) && al16(v) && (long long)D.B * D.Hkv * D.L < (1ll << 31);
 }
 
-// The number of CTAs per (b, KV group): as many as two per SM allow, at most one per tile.
+// The number of CTAs per (b, KV group, query): as many as two per SM allow, at most one per tile and at
+// most 16 (so the last CTA merges few partials: at small batches a split is then 2-3 tiles).
 int decode_attn_mma_splits(const Dims &D, int ntiles) {
-    const int per_bg = std::max(1, (kCtasPerSm * num_sms()) / std::max(1, D.B * D.Hkv));
-    return std::max(1, std::min(per_bg, ntiles));
+    const int per_bg = std::max(1, (kCtasPerSm * num_sms()) / std::max(1, D.B * D.Hkv * D.T));
+    return std::max(1, std::min(std::min(per_bg, ntiles), 16));
 }
 
 unsigned int decode_attn_mma_error_flags(bool clear) {
@@ -332,7 +341,7 @@ unsigned int decode_attn_mma_error_flags(bool clear) {
     return v;
 }
 
-// `partial` holds B * Hq * nsplit * 132 floats (16-byte aligned); `counters` B * Hkv zeros.
+// `partial` holds B * Hq * T * nsplit * 132 floats (16-byte aligned); `counters` B * Hkv * T zeros.
 cudaError_t launch_decode_attn_mma(const Dims &D, int n, int ntiles, const void *q, const void *k_cache,
                                    const void *v_cache, const float *scores, const int *sel, float *partial,
                                    unsigned int *counters, void *out, float *lse, cudaStream_t stream) {
@@ -343,7 +352,7 @@ cudaError_t launch_decode_attn_mma(const Dims &D, int n, int ntiles, const void 
     const size_t smem = 1024 + kStages * 2 * kTileBytes;
     cudaFuncSetAttribute(decode_attn_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     const int nsplit = decode_attn_mma_splits(D, ntiles);
-    decode_attn_mma_kernel<<<dim3(nsplit, D.Hkv, D.B), kThreads, smem, stream>>>(
+    decode_attn_mma_kernel<<<dim3(nsplit, D.Hkv, D.B * D.T), kThreads, smem, stream>>>(
         kmap, vmap, D, n, ntiles, (const __nv_bfloat16 *)q, scores, sel, partial, counters, (__nv_bfloat16 *)out,
         lse);
     return cudaGetLastError();

@@ -12,6 +12,8 @@ namespace hils {
 
 size_t bwd_smem_bytes(const Dims &D);
 bool decode_supported(const Dims &D);
+bool decode_multi_supported(const Dims &D, int dtype, const void *q, const void *q_hat, const void *k, const void *v,
+                            const void *k_sum);
 cudaError_t launch_attn_fwd_simt(const Dims &D, int dtype, const void *q, const void *k, const void *v,
                                  const void *q_hat, const void *k_sum, const float *b_sum, const int *idx, void *out,
                                  float *lse, cudaStream_t stream);
@@ -226,8 +228,8 @@ hils_status hils_decode(const hils_params *p, const void *q, const void *q_hat, 
     Dims D;
     hils_status st = resolve(p, fn, &D);
     if (st != HILS_OK) return st;
-    if (D.T != 1 || D.q_pos0 != D.L - 1)
-        return fail(HILS_ERR_INVALID_ARG, "%s: needs T == 1 and q_pos0 == L-1 (got T=%d q_pos0=%d L=%d)", fn, D.T,
+    if (D.T < 1 || D.T > 8 || D.q_pos0 != D.L - D.T)
+        return fail(HILS_ERR_INVALID_ARG, "%s: needs 1 <= T <= 8 and q_pos0 == L-T (got T=%d q_pos0=%d L=%d)", fn, D.T,
                     D.q_pos0, D.L);
     HILS_REQUIRE_PTR(q);
     HILS_REQUIRE_PTR(q_hat);
@@ -245,6 +247,9 @@ hils_status hils_decode(const hils_params *p, const void *q, const void *q_hat, 
     if (!decode_supported(D))
         return fail(HILS_ERR_UNSUPPORTED, "%s: %d candidate chunks with G=%d, topk=%d exceed the selection buffers", fn,
                     D.Nc, D.G, D.topk);
+    if (!decode_multi_supported(D, p->dtype, q, q_hat, k_cache, v_cache, k_sum))
+        return fail(HILS_ERR_UNSUPPORTED, "%s: T=%d > 1 needs bf16, d 128, S 64, G <= 8, topk <= 32 and 16-byte "
+                    "aligned q, q_hat, caches and k_sum", fn, D.T);
     st = check_ws(fn, workspace, workspace_bytes, decode_workspace_bytes(D));
     if (st != HILS_OK) return st;
     return cuda_status(launch_decode(D, p->dtype, q, q_hat, k_cache, v_cache, k_sum, b_sum, out, lse, idx_out, workspace,

@@ -198,26 +198,33 @@ def attn_fwd(q, k, v, q_hat, k_sum, b_sum, idx, *, S: int, window: int, q_pos0: 
 
 def decode(q, q_hat, k_cache, v_cache, k_sum, b_sum, *, S: int, topk: int, window: int, scale: float = 0.0,
            out=None, lse=None, idx_out=None, return_idx: bool = False, workspace=None):
-    """One decode step at position L-1. q, q_hat [B,Hq,1,d]; caches [B,Hkv,L,d]; k_sum [B,Hq,Nc,d]; b_sum
-    [B,Hq,Nc] -> out [B,Hq,1,d], lse [B,Hq] (and idx [B,Hkv,topk] with return_idx)."""
-    B, Hq, T, d = q.shape
+    """One decode step for the last M = q.shape[2] positions of the cache (M = 1: position L-1).
+    q, q_hat [B,Hq,M,d]; caches [B,Hkv,L,d]; k_sum [B,Hq,Nc,d]; b_sum [B,Hq,Nc] -> out [B,Hq,M,d],
+    lse [B,Hq] for M = 1 else [B,Hq,M] (and idx [B,Hkv,topk] for M = 1 else [B,Hkv,M,topk] with
+    return_idx)."""
+    B, Hq, M, d = q.shape
     Hkv, L = k_cache.shape[1], k_cache.shape[2]
     dev, dt = q.device, q.dtype
     Nc = L // S
-    _check("q_hat", q_hat, dt, (B, Hq, 1, d), dev)
+    _check("q", q, dt, (B, Hq, M, d), dev)
+    _check("q_hat", q_hat, dt, (B, Hq, M, d), dev)
     _check("k_cache", k_cache, dt, (B, Hkv, L, d), dev)
     _check("v_cache", v_cache, dt, (B, Hkv, L, d), dev)
     _check("k_sum", k_sum, dt, (B, Hq, Nc, d), dev)
     _check("b_sum", b_sum, torch.float32, (B, Hq, Nc), dev)
+    lse_shape = (B, Hq) if M == 1 else (B, Hq, M)
+    idx_shape = (B, Hkv, topk) if M == 1 else (B, Hkv, M, topk)
     if out is None:
-        out = torch.empty((B, Hq, 1, d), dtype=dt, device=dev)
+        out = torch.empty((B, Hq, M, d), dtype=dt, device=dev)
     if lse is None:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=dev)
+    _check("out", out, dt, (B, Hq, M, d), dev)
+    _check("lse", lse, torch.float32, lse_shape, dev)
     if return_idx and idx_out is None:
-        idx_out = torch.empty((B, Hkv, topk), dtype=torch.int32, device=dev)
+        idx_out = torch.empty(idx_shape, dtype=torch.int32, device=dev)
     if idx_out is not None:
-        _check("idx_out", idx_out, torch.int32, (B, Hkv, topk), dev)
-    p = make_params(B, 1, L, Hq, Hkv, d, S, topk, window, L - 1, scale, dt)
+        _check("idx_out", idx_out, torch.int32, idx_shape, dev)
+    p = make_params(B, M, L, Hq, Hkv, d, S, topk, window, L - M, scale, dt)
     ws, nws = _workspace(p, OP_DECODE, dev, workspace)
     _raise(lib.hils_decode(ctypes.byref(p), _ptr(q), _ptr(q_hat), _ptr(k_cache), _ptr(v_cache), _ptr(k_sum),
                            _ptr(b_sum), _ptr(out), _ptr(lse), _ptr(idx_out), _ptr(ws), nws, _stream(dev)))

@@ -114,14 +114,16 @@ def prefill_inputs(w: Workload, seed: int = 0, device="cpu", with_dout: bool = F
 
 
 def decode_inputs(w: Workload, seed: int = 0, device="cpu") -> dict:
-    """Needle-in-a-haystack decode cache. q, q_hat [B,Hq,1,d]; k_cache, v_cache [B,Hkv,L,d];
-    q_land [B,Hq,Nc,d]; needle_chunks [B,needles] (int64, the planted chunk ids).
+    """Needle-in-a-haystack decode cache for the last M = w.T positions (M = 1: plain decode; M > 1:
+    multi-token decode). q, q_hat [B,Hq,M,d]; k_cache, v_cache [B,Hkv,L,d]; q_land [B,Hq,Nc,d];
+    needle_chunks [B,needles] (int64, the planted chunk ids, candidates of the last query; the needle
+    keys follow the first query token's q^).
     The cache is filled one sequence at a time so that only one fp32 slice is live at once."""
-    assert w.T == 1 and w.q_pos0 == w.L - 1
+    assert 1 <= w.T and w.q_pos0 == w.L - w.T
     g = _gen(seed, device)
     B, L, Hq, Hkv, d, S, G = w.B, w.L, w.Hq, w.Hkv, w.d, w.S, w.G
     dt = w.torch_dtype
-    q = _randn((B, Hq, 1, d), g, device)
+    q = _randn((B, Hq, w.T, d), g, device)
     q_land = _randn((B, Hq, w.Nc, d), g, device)
     q_hat = _qcal(q, d, g, device)
     left = max(0, L - 1 - w.W + 1) // S * S

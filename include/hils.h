@@ -125,10 +125,14 @@ HILS_API hils_status hils_attn_fwd(const hils_params *p, const void *q, const vo
                           void *workspace, size_t workspace_bytes, hils_stream_t stream);
 
 /*
- * One decode step (stages b-d for T = 1 at position q_pos0 = L-1 over a KV cache of L tokens):
- * scores every candidate chunk's summary, selects topk chunks per KV group as hils_select_topk
- * does, attends, and fuses as hils_attn_fwd does. q, q_hat [B, Hq, 1, d]; out [B, Hq, 1, d];
- * lse [B, Hq]; idx_out (nullable) [B, Hkv, topk]. Requires T == 1 and q_pos0 == L-1.
+ * One decode step (stages b-d) for T = M query tokens per sequence at positions q_pos0 .. L-1 with
+ * q_pos0 = L-M (M = 1: the usual single-token step; 2 <= M <= 8: multi-token decode, e.g. verifying M
+ * speculated tokens, each query with its own window and selection) over a KV cache of L tokens that
+ * already holds them: scores every candidate chunk's summary (each summary row read once for all M
+ * queries), selects topk chunks per KV group and query as hils_select_topk does, attends, and fuses
+ * as hils_attn_fwd does. q, q_hat [B, Hq, M, d]; out [B, Hq, M, d]; lse [B, Hq, M]; idx_out (nullable)
+ * [B, Hkv, M, topk]. M > 1 needs bf16, d 128, S 64, G <= 8, topk <= 32 and 16-byte aligned q, q_hat,
+ * caches and k_sum (HILS_ERR_UNSUPPORTED otherwise).
  * Workspace: hils_workspace_size(p, HILS_OP_DECODE) bytes.
  */
 HILS_API hils_status hils_decode(const hils_params *p, const void *q, const void *q_hat, const void *k_cache,

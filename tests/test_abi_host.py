@@ -78,7 +78,7 @@ def test_null_and_misaligned_pointers():
 def test_decode_and_bwd_shape_rules():
     p = P(T=1, q_pos0=10)
     st = H.lib.hils_decode(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None)
-    assert st == 1 and b"q_pos0 == L-1" in H.lib.hils_last_error()
+    assert st == 1 and b"q_pos0 == L-T" in H.lib.hils_last_error()
     p = P(T=1, q_pos0=255)
     st = H.lib.hils_decode(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 16, None)
     assert st == 3  # workspace too small
@@ -86,6 +86,27 @@ def test_decode_and_bwd_shape_rules():
     args = [FAKE] * 17
     st = H.lib.hils_attn_bwd(ctypes.byref(p), *args, 1 << 30, None)
     assert st == 1 and b"self-attention" in H.lib.hils_last_error()
+
+
+def test_multi_token_decode_rules():
+    # M = T query tokens at the end of the cache: 1 <= M <= 8 and q_pos0 == L - M
+    p = P(T=9, q_pos0=256 - 9)
+    st = H.lib.hils_decode(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None)
+    assert st == 1 and b"T <= 8" in H.lib.hils_last_error()
+    p = P(T=4, q_pos0=256 - 3)
+    st = H.lib.hils_decode(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None)
+    assert st == 1
+    # M > 1 runs on the bf16 d 128 S 64 kernels only
+    p = P(T=4, q_pos0=256 - 4, dtype=1)
+    st = H.lib.hils_decode(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None)
+    assert st == 2 and b"T=4 > 1 needs bf16" in H.lib.hils_last_error()
+    # supported shape: the workspace grows with M
+    one, four = P(T=1, L=65536, q_pos0=65535), P(T=4, L=65536, q_pos0=65532)
+    n1 = H.lib.hils_workspace_size(ctypes.byref(one), H.OP_DECODE)
+    n4 = H.lib.hils_workspace_size(ctypes.byref(four), H.OP_DECODE)
+    assert n4 > 3 * n1 // 2
+    st = H.lib.hils_decode(ctypes.byref(four), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 16, None)
+    assert st == 3  # workspace too small: everything before it validated
 
 
 def test_summary_range_checked():

@@ -135,3 +135,59 @@ def test_decode_select_periodic_scores():
     ro, rl = oracle.attn_fwd(g1, np64(x["q"]), np64(x["k_cache"]), np64(x["v_cache"]), qh, rk, rb, ridx)
     assert_close(out, ro, TOL["bf16"], "periodic out")
     assert_close(lse, rl[..., 0], TOL["bf16"], "periodic lse")
+
+
+@pytest.mark.parametrize("w", [
+    # positions 4093..4096 with W 256: the window's left edge crosses a chunk boundary inside the block,
+    # so the queries have 59, 59, 60 and 60 candidates
+    W.Workload("dec_m4_straddle", B=2, T=4, L=4097, Hq=8, Hkv=2, d=128, S=64, topk=8, W=256, dtype="bf16",
+               recipe="needle", q_pos0=4093, needles=4),
+    W.Workload("dec_m8_g8", B=1, T=8, L=5000, Hq=16, Hkv=2, d=128, S=64, topk=12, W=300, dtype="bf16",
+               recipe="needle", q_pos0=4992, needles=5),
+    W.Workload("dec_m2_g1", B=3, T=2, L=3000, Hq=4, Hkv=4, d=128, S=64, topk=8, W=200, dtype="bf16",
+               recipe="needle", q_pos0=2998, needles=3),
+], ids=lambda w: w.name)
+def test_multi_token_decode(w):
+    """M query tokens at the end of the cache in one decode call: per query its own candidates, top-k
+    and window, equal to the oracle's prefill-form evaluation of the same M rows."""
+    x = W.decode_inputs(w, seed=3, device="cpu")
+    xd = {n: t.cuda() for n, t in x.items()}
+    k_sum, b_sum = H.chunk_summary(xd["k_cache"], xd["q_land"], w.S)
+    out, lse, idx = H.decode(xd["q"], xd["q_hat"], xd["k_cache"], xd["v_cache"], k_sum, b_sum, S=w.S, topk=w.topk,
+                             window=w.W, return_idx=True)
+    assert tuple(out.shape) == (w.B, w.Hq, w.T, w.d) and tuple(lse.shape) == (w.B, w.Hq, w.T)
+    assert tuple(idx.shape) == (w.B, w.Hkv, w.T, w.topk)
+    tol = TOL[w.dtype]
+    for b in range(w.B):
+        for grp in range(w.Hkv):
+            hs = slice(grp * w.G, (grp + 1) * w.G)
+            g1 = Geometry(B=1, T=w.T, L=w.L, Hq=w.G, Hkv=1, d=w.d, S=w.S, topk=w.topk, W=w.W, q_pos0=w.q_pos0)
+            kk = np64(x["k_cache"][b:b + 1, grp:grp + 1])
+            vv = np64(x["v_cache"][b:b + 1, grp:grp + 1])
+            rk, rb = oracle.chunk_summary(g1, kk, np64(x["q_land"][b:b + 1, hs]))
+            qh = np64(x["q_hat"][b:b + 1, hs])
+            ridx, rgap = oracle.select_topk(g1, qh, rk, rb)
+            near = check_idx(idx[b:b + 1, grp:grp + 1], ridx, rgap, f"multi idx b{b} g{grp}")
+            if near.any():
+                continue
+            ro, rl = oracle.attn_fwd(g1, np64(x["q"][b:b + 1, hs]), kk, vv, qh, rk, rb, ridx)
+            assert_close(out[b:b + 1, hs], ro, tol, f"multi out b{b} g{grp}")
+            assert_close(lse[b:b + 1, hs], np.asarray(rl).reshape(1, w.G, w.T), tol, f"multi lse b{b} g{grp}")
+
+
+def test_multi_token_decode_rows_match_single_token_at_last_position():
+    """The last of M queries sees exactly what a single-token step at L-1 sees (same cache, same row)."""
+    w = W.Workload("dec_m4_vs_m1", B=2, T=4, L=6000, Hq=8, Hkv=2, d=128, S=64, topk=16, W=512, dtype="bf16",
+                   recipe="needle", q_pos0=5996, needles=6)
+    x = {n: t.cuda() for n, t in W.decode_inputs(w, seed=9, device="cpu").items()}
+    k_sum, b_sum = H.chunk_summary(x["k_cache"], x["q_land"], w.S)
+    out4, lse4, idx4 = H.decode(x["q"], x["q_hat"], x["k_cache"], x["v_cache"], k_sum, b_sum, S=w.S, topk=w.topk,
+                                window=w.W, return_idx=True)
+    q1, qh1 = x["q"][:, :, 3:].contiguous(), x["q_hat"][:, :, 3:].contiguous()
+    out1, lse1, idx1 = H.decode(q1, qh1, x["k_cache"], x["v_cache"], k_sum, b_sum, S=w.S, topk=w.topk, window=w.W,
+                                return_idx=True)
+    # the two paths score with different kernels (fp32 sums in different orders): same ids, outputs
+    # within a couple of bf16 steps
+    assert torch.equal(idx4[:, :, 3], idx1)
+    assert torch.allclose(out4[:, :, 3:].float(), out1.float(), atol=1e-2, rtol=0)
+    assert torch.allclose(lse4[:, :, 3], lse1, atol=1e-3, rtol=0)
