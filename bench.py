@@ -221,21 +221,26 @@ def prefill_work(w: W.Workload):
             "avg_attended": attended / w.T}
 
 
-def decode_bytes(w: W.Workload):
+def decode_bytes(w: W.Workload, idx=None):
     """Bytes one decode step must touch for its M = w.T queries at the end of the cache: every candidate
-    summary once (k' in the input dtype + fp32 b'; the last query's candidates, the most), and per query
-    its selected chunks' K and V, its window's K and V, and q, q^ and the output."""
+    summary once (k' in the input dtype + fp32 b'; the last query's candidates, the most), the K and V
+    of the selected chunks and of the window, and q, q^ and the output. With M > 1 the queries of a
+    KV group share what they touch: chunks count once per group over the union of the M selections
+    (`idx` [B, Hkv, M, topk] of one step; without it, the per-query sum is an upper bound) and the
+    window is the union of the M windows, tokens l_(L-M) .. L-1."""
     el = 2 if w.dtype == "bf16" else 4
     M = w.T
     p_last = w.L - 1
     n_last = window_left(p_last, w.W, w.S) // w.S
     summ = w.B * w.Hq * n_last * (w.d * el + 4)
-    chunks = win = 0
-    for m in range(M):
-        p = w.L - M + m
-        l = window_left(p, w.W, w.S)
-        chunks += w.B * w.Hkv * min(w.topk, l // w.S) * w.S * w.d * el * 2
-        win += w.B * w.Hkv * (p - l + 1) * w.d * el * 2
+    tile = w.S * w.d * el * 2
+    if M > 1 and idx is not None:
+        ids = idx.reshape(w.B * w.Hkv, M * w.topk).cpu()
+        chunks = sum(len(set(r.tolist()) - {-1}) for r in ids) * tile
+    else:
+        chunks = sum(w.B * w.Hkv * min(w.topk, window_left(w.L - M + m, w.W, w.S) // w.S) * tile
+                     for m in range(M))
+    win = w.B * w.Hkv * (w.L - window_left(w.L - M, w.W, w.S)) * w.d * el * 2
     io = w.B * w.Hq * M * (w.d * el * 3 + 4)
     return {"total": summ + chunks + win + io, "summaries": summ, "chunks": chunks, "window": win, "io": io}
 
@@ -373,7 +378,7 @@ def bench_decode(args, dist, dev, H, peaks, w: W.Workload, steps: int):
         first = idx[b, 0] if w.T == 1 else idx[b, 0, 0]  # the needle keys follow the first query's q^
         needles_found += len(set(x["needle_chunks"][b].tolist()) & set(first.tolist()))
     ms_step = dist.max(total_ms / steps)  # per-sequence-batch latency: the slowest rank's
-    nbytes = decode_bytes(w)
+    nbytes = decode_bytes(w, idx)
     gbs = nbytes["total"] / (ms_step / 1e3) / 1e9
     del graph
     summ = {"ms": summ_ms, "bytes": summ_bytes, "achieved_gbs": summ_bytes / (summ_ms / 1e3) / 1e9,

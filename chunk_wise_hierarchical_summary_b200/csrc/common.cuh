@@ -19,6 +19,12 @@ struct Dims {
     float tau;
 };
 
+// Row of the landmark query used for (b, query head h, chunk c): q_land [B, Hq, Nc, d], or with a
+// shared query (one learned vector per head, Sec. 4 "landmark tokens" alternative) q_land [Hq, d].
+__host__ __device__ __forceinline__ size_t landmark_row(const Dims &D, int shared_q, int b, int h, int c) {
+    return shared_q ? (size_t)h : ((size_t)b * D.Hq + h) * D.Nc + c;
+}
+
 __host__ __device__ __forceinline__ int window_left(int pos, int W, int S) {
     int e = pos - W + 1;
     if (e < 0) e = 0;

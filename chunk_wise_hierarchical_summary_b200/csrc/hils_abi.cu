@@ -152,9 +152,11 @@ size_t hils_workspace_size(const hils_params *p, int op) {
     }
 }
 
-hils_status hils_chunk_summary(const hils_params *p, const void *k, const void *q_land, int32_t c_begin,
-                               int32_t c_end, void *k_sum, float *b_sum, hils_stream_t stream) {
-    const char *fn = "hils_chunk_summary";
+namespace {
+
+hils_status chunk_summary_common(const char *fn, const hils_params *p, const void *k, const void *q_land,
+                                 bool shared_q, int32_t c_begin, int32_t c_end, void *k_sum, float *b_sum,
+                                 hils_stream_t stream) {
     Dims D;
     hils_status st = resolve(p, fn, &D);
     if (st != HILS_OK) return st;
@@ -162,12 +164,30 @@ hils_status hils_chunk_summary(const hils_params *p, const void *k, const void *
         return fail(HILS_ERR_INVALID_ARG, "%s: chunk range [%d, %d) outside [0, %d]", fn, c_begin, c_end, D.Nc);
     if (c_end == c_begin) return HILS_OK;  // empty range: nothing is read or written
     HILS_REQUIRE_PTR(k);
-    HILS_REQUIRE_PTR(q_land);
+    {
+        const char *qn = shared_q ? "q_shared" : "q_land";
+        if (q_land == nullptr) return fail(HILS_ERR_INVALID_ARG, "%s: %s is NULL", fn, qn);
+        if (!aligned16(q_land)) return fail(HILS_ERR_INVALID_ARG, "%s: %s is not 16-byte aligned", fn, qn);
+    }
     HILS_REQUIRE_PTR(k_sum);
     HILS_REQUIRE_PTR(b_sum);
     if (D.Hkv > 65535) return fail(HILS_ERR_UNSUPPORTED, "%s: Hkv must be <= 65535", fn);
-    return cuda_status(launch_chunk_summary(D, p->dtype, k, q_land, c_begin, c_end, k_sum, b_sum, (cudaStream_t)stream),
-                       fn);
+    return cuda_status(
+        launch_chunk_summary(D, p->dtype, k, q_land, shared_q, c_begin, c_end, k_sum, b_sum, (cudaStream_t)stream), fn);
+}
+
+}  // namespace
+
+hils_status hils_chunk_summary(const hils_params *p, const void *k, const void *q_land, int32_t c_begin,
+                               int32_t c_end, void *k_sum, float *b_sum, hils_stream_t stream) {
+    return chunk_summary_common("hils_chunk_summary", p, k, q_land, false, c_begin, c_end, k_sum, b_sum, stream);
+}
+
+hils_status hils_chunk_summary_shared_query(const hils_params *p, const void *k, const void *q_shared,
+                                            int32_t c_begin, int32_t c_end, void *k_sum, float *b_sum,
+                                            hils_stream_t stream) {
+    return chunk_summary_common("hils_chunk_summary_shared_query", p, k, q_shared, true, c_begin, c_end, k_sum, b_sum,
+                                stream);
 }
 
 hils_status hils_select_topk(const hils_params *p, const void *q_hat, const void *k_sum, const float *b_sum,

@@ -9,8 +9,8 @@
 namespace hils {
 
 // Each launcher enqueues its kernels on `stream` and returns the launch status.
-cudaError_t launch_chunk_summary(const Dims &D, int dtype, const void *k, const void *q_land, int c_begin,
-                                 int c_end, void *k_sum, float *b_sum, cudaStream_t stream);
+cudaError_t launch_chunk_summary(const Dims &D, int dtype, const void *k, const void *q_land, bool shared_q,
+                                 int c_begin, int c_end, void *k_sum, float *b_sum, cudaStream_t stream);
 
 size_t select_smem_bytes(const Dims &D);
 cudaError_t launch_select_topk(const Dims &D, int dtype, const void *q_hat, const void *k_sum, const float *b_sum,

@@ -16,8 +16,8 @@ constexpr int kSummaryWarps = 4;
 
 template <typename T>
 __global__ void __launch_bounds__(kSummaryWarps * 32)
-summary_kernel(Dims D, const T *__restrict__ k, const T *__restrict__ q_land, int c_begin, T *__restrict__ k_sum,
-               float *__restrict__ b_sum) {
+summary_kernel(Dims D, const T *__restrict__ k, const T *__restrict__ q_land, int shared_q, int c_begin,
+               T *__restrict__ k_sum, float *__restrict__ b_sum) {
     extern __shared__ float smem[];
     const int c = c_begin + blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int d = D.d, S = D.S, G = D.G;
@@ -38,7 +38,7 @@ summary_kernel(Dims D, const T *__restrict__ k, const T *__restrict__ q_land, in
     for (int e = threadIdx.x * 8; e < G * d; e += blockDim.x * 8) {
         const int hh = e / d, t = e % d;
         float f[8];
-        load8(q_land + (((size_t)b * D.Hq + g * G + hh) * D.Nc + c) * d + t, f);
+        load8(q_land + landmark_row(D, shared_q, b, g * G + hh, c) * d + t, f);
 #pragma unroll
         for (int u = 0; u < 8; ++u) qs[e + u] = f[u];
     }
@@ -87,26 +87,26 @@ summary_kernel(Dims D, const T *__restrict__ k, const T *__restrict__ q_land, in
 }  // namespace
 
 bool summary_mma_supported(const Dims &D, int dtype, const void *k, const void *q_land, const void *k_sum);
-cudaError_t launch_summary_mma(const Dims &D, const void *k, const void *q_land, int c_begin, int c_end,
-                               void *k_sum, float *b_sum, cudaStream_t stream);
+cudaError_t launch_summary_mma(const Dims &D, const void *k, const void *q_land, bool shared_q, int c_begin,
+                               int c_end, void *k_sum, float *b_sum, cudaStream_t stream);
 
-cudaError_t launch_chunk_summary(const Dims &D, int dtype, const void *k, const void *q_land, int c_begin, int c_end,
-                                 void *k_sum, float *b_sum, cudaStream_t stream) {
+cudaError_t launch_chunk_summary(const Dims &D, int dtype, const void *k, const void *q_land, bool shared_q,
+                                 int c_begin, int c_end, void *k_sum, float *b_sum, cudaStream_t stream) {
     if (c_end <= c_begin) return cudaSuccess;
     if (summary_mma_supported(D, dtype, k, q_land, k_sum))
-        return launch_summary_mma(D, k, q_land, c_begin, c_end, k_sum, b_sum, stream);
+        return launch_summary_mma(D, k, q_land, shared_q, c_begin, c_end, k_sum, b_sum, stream);
     const size_t smem = sizeof(float) * ((size_t)D.S * (D.d + 1) + (size_t)D.G * D.d + (size_t)kSummaryWarps * D.S);
     dim3 grid(c_end - c_begin, D.Hkv, D.B);
     if (dtype == HILS_BF16) {
         auto kern = summary_kernel<__nv_bfloat16>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         kern<<<grid, kSummaryWarps * 32, smem, stream>>>(D, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)q_land,
-                                                         c_begin, (__nv_bfloat16 *)k_sum, b_sum);
+                                                         (int)shared_q, c_begin, (__nv_bfloat16 *)k_sum, b_sum);
     } else {
         auto kern = summary_kernel<float>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        kern<<<grid, kSummaryWarps * 32, smem, stream>>>(D, (const float *)k, (const float *)q_land, c_begin,
-                                                         (float *)k_sum, b_sum);
+        kern<<<grid, kSummaryWarps * 32, smem, stream>>>(D, (const float *)k, (const float *)q_land,
+                                                         (int)shared_q, c_begin, (float *)k_sum, b_sum);
     }
     return cudaGetLastError();
 }

@@ -40,7 +40,7 @@ __device__ unsigned int g_summary_errors = 0;
 
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 summary_mma_kernel(const __grid_constant__ CUtensorMap kmap, Dims D, const __nv_bfloat16 *__restrict__ q_land,
-                   int c_begin, int nc, __nv_bfloat16 *__restrict__ k_sum, float *__restrict__ b_sum) {
+                   int shared_q, int c_begin, int nc, __nv_bfloat16 *__restrict__ k_sum, float *__restrict__ b_sum) {
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
     __shared__ float red_m[kConsumerWarps][8], red_z[kConsumerWarps][8], red_e[kConsumerWarps][8];
@@ -81,7 +81,7 @@ summary_mma_kernel(const __grid_constant__ CUtensorMap kmap, Dims D, const __nv_
                 tma_load_2d(Kt, &kmap, 0, y, &full[st]);
                 tma_load_2d(Kt + 8192, &kmap, 64, y, &full[st]);
                 for (int h = 0; h < G; ++h)
-                    bulk_g2s(Qt + h * kQRowBytes, q_land + (((size_t)b * D.Hq + g * G + h) * D.Nc + c) * 128, 256,
+                    bulk_g2s(Qt + h * kQRowBytes, q_land + landmark_row(D, shared_q, b, g * G + h, c) * 128, 256,
                              &full[st]);
             }
         }
@@ -238,8 +238,8 @@ unsigned int summary_error_flags(bool clear) {
     return v;
 }
 
-cudaError_t launch_summary_mma(const Dims &D, const void *k, const void *q_land, int c_begin, int c_end,
-                               void *k_sum, float *b_sum, cudaStream_t stream) {
+cudaError_t launch_summary_mma(const Dims &D, const void *k, const void *q_land, bool shared_q, int c_begin,
+                               int c_end, void *k_sum, float *b_sum, cudaStream_t stream) {
     const int nc = c_end - c_begin;
     if (nc <= 0) return cudaSuccess;
     CUtensorMap kmap;
@@ -248,7 +248,8 @@ cudaError_t launch_summary_mma(const Dims &D, const void *k, const void *q_land,
     cudaFuncSetAttribute(summary_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     const long long units = (long long)nc * D.Hkv * D.B;
     const int grid = (int)std::min<long long>(units, (long long)kCtasPerSm * num_sms());
-    summary_mma_kernel<<<grid, kThreads, smem, stream>>>(kmap, D, (const __nv_bfloat16 *)q_land, c_begin, nc,
+    summary_mma_kernel<<<grid, kThreads, smem, stream>>>(kmap, D, (const __nv_bfloat16 *)q_land, (int)shared_q,
+                                                         c_begin, nc,
                                                          (__nv_bfloat16 *)k_sum, b_sum);
     return cudaGetLastError();
 }

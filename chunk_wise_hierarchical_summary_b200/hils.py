@@ -26,9 +26,9 @@ HILS_BF16, HILS_FP32 = 0, 1
 OP_SUMMARY, OP_SELECT, OP_ATTN_FWD, OP_DECODE, OP_ATTN_BWD = 0, 1, 2, 3, 4
 
 # Every symbol include/hils.h declares (checked by the tests against the header and the library).
-EXPORTED = ("hils_workspace_size", "hils_chunk_summary", "hils_select_topk", "hils_attn_fwd", "hils_decode",
-            "hils_attn_bwd", "hils_check", "hils_status_string", "hils_last_error", "hils_version",
-            "hils_decode_noalloc")
+EXPORTED = ("hils_workspace_size", "hils_chunk_summary", "hils_chunk_summary_shared_query", "hils_select_topk",
+            "hils_attn_fwd", "hils_decode", "hils_attn_bwd", "hils_check", "hils_status_string", "hils_last_error",
+            "hils_version", "hils_decode_noalloc")
 
 
 class HilsError(RuntimeError):
@@ -52,6 +52,8 @@ def _load() -> ctypes.CDLL:
     lib.hils_workspace_size.restype = ctypes.c_size_t
     lib.hils_chunk_summary.argtypes = [P, vp, vp, ctypes.c_int32, ctypes.c_int32, vp, vp, vp]
     lib.hils_chunk_summary.restype = st
+    lib.hils_chunk_summary_shared_query.argtypes = [P, vp, vp, ctypes.c_int32, ctypes.c_int32, vp, vp, vp]
+    lib.hils_chunk_summary_shared_query.restype = st
     lib.hils_select_topk.argtypes = [P, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.hils_select_topk.restype = st
     lib.hils_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
@@ -144,6 +146,28 @@ def chunk_summary(k, q_land, S: int, *, c_begin: int = 0, c_end: int | None = No
     c_end = Nc if c_end is None else c_end
     _raise(lib.hils_chunk_summary(ctypes.byref(p), _ptr(k), _ptr(q_land), c_begin, c_end, _ptr(k_sum), _ptr(b_sum),
                                   _stream(dev)))
+    return k_sum, b_sum
+
+
+def chunk_summary_shared_query(k, q_shared, S: int, *, c_begin: int = 0, c_end: int | None = None, k_sum=None,
+                               b_sum=None, scale: float = 0.0):
+    """Eq. 8 summaries with one shared landmark query per head (Sec. 4): k [B,Hkv,L,d], q_shared [Hq,d]
+    -> (k_sum [B,Hq,Nc,d], b_sum [B,Hq,Nc] fp32), as chunk_summary with q_land[b,h,c] = q_shared[h]."""
+    B, Hkv, L, d = k.shape
+    Hq, Nc = q_shared.shape[0], L // S
+    dev, dt = k.device, k.dtype
+    _check("q_shared", q_shared, dt, (Hq, d), dev)
+    if k_sum is None:
+        k_sum = torch.empty((B, Hq, Nc, d), dtype=dt, device=dev)
+    if b_sum is None:
+        b_sum = torch.empty((B, Hq, Nc), dtype=torch.float32, device=dev)
+    _check("k_sum", k_sum, dt, (B, Hq, Nc, d), dev)
+    _check("b_sum", b_sum, torch.float32, (B, Hq, Nc), dev)
+    _check("k", k, dt, (B, Hkv, L, d), dev)
+    p = make_params(B, 1, L, Hq, Hkv, d, S, 1, 1, 0, scale, dt)
+    c_end = Nc if c_end is None else c_end
+    _raise(lib.hils_chunk_summary_shared_query(ctypes.byref(p), _ptr(k), _ptr(q_shared), c_begin, c_end, _ptr(k_sum),
+                                               _ptr(b_sum), _stream(dev)))
     return k_sum, b_sum
 
 

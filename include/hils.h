@@ -97,6 +97,17 @@ HILS_API hils_status hils_chunk_summary(const hils_params *p, const void *k, con
                                int32_t c_end, void *k_sum, float *b_sum, hils_stream_t stream);
 
 /*
+ * Stage (a) with the shared landmark query (Sec. 4, the alternative to landmark tokens: one learned
+ * query vector per head and layer instead of one per chunk): exactly hils_chunk_summary with
+ * q_land[b,h,c] := q_shared[h] for every b and c. q_shared [Hq, d] in params.dtype (16-byte aligned
+ * for the bf16 fast path); every other argument, layout, range rule and error as hils_chunk_summary.
+ * Forward only: the gradient for q_shared is the sum over (b, c) of hils_attn_bwd's dq_land.
+ */
+HILS_API hils_status hils_chunk_summary_shared_query(const hils_params *p, const void *k, const void *q_shared,
+                                                     int32_t c_begin, int32_t c_end, void *k_sum, float *b_sum,
+                                                     hils_stream_t stream);
+
+/*
  * Stage (b), Eq. 7 + Sec. 3 RQ1 + Sec. 4 "GQA": for every (b, KV group g, row i) with n = n_p
  * candidates:  s^_{h,c} = tau * q_hat[b,h,i] . k_sum[b,h,c] + b_sum[b,h,c]  for c < n and each head h
  * of the group; group score g_c = max_h (s^_{h,c} - LSE_{c'<n} s^_{h,c'}); keep the min(topk, n)

@@ -6,6 +6,7 @@ CPU-baseline leg. The product path (the CUDA library and its Python binding) nev
 Every function converts its inputs to contiguous fp64 (int32 for idx) and calls the plain C
 statement in hils_oracle.c, which cites the paper section / equation each step follows:
   chunk_summary  Eq. 8 (Prop. 3.1)            select_topk  Sec. 3 RQ1 + Sec. 4 GQA selection
+  chunk_summary_shared_query  Eq. 8 with one landmark query per head (Sec. 4)
   attn_fwd       Eq. 10, chunked form          eq10_tokenwise  Eq. 10, token by token
   attn_bwd       gradients of the above with the selection held fixed
   decode         select_topk + attn_fwd for one query at position L-1
@@ -136,6 +137,14 @@ def chunk_summary(g: Geometry, k, q_land, c_begin: int = 0, c_end: int | None = 
     bs = np.zeros((g.B, g.Hq, g.Nc))
     _load().orc_chunk_summary(ctypes.byref(g._c()), _pd(k), _pd(ql), int(c_begin), int(c_end), _pd(ks), _pd(bs))
     return ks, bs
+
+
+def chunk_summary_shared_query(g: Geometry, k, q_shared, c_begin: int = 0, c_end: int | None = None):
+    """Eq. 8 with the shared landmark query of Sec. 4 (one learned query per head instead of one per
+    chunk): the summary of chunk c of sequence b under head h uses q_shared[h] as its landmark query."""
+    qs = _f64(q_shared, (g.Hq, g.d))
+    q_land = np.broadcast_to(qs[None, :, None, :], (g.B, g.Hq, g.Nc, g.d))
+    return chunk_summary(g, k, q_land, c_begin, c_end)
 
 
 def select_topk(g: Geometry, q_hat, k_sum, b_sum):

@@ -115,6 +115,15 @@ def test_summary_range_checked():
     assert st == 1 and b"chunk range" in H.lib.hils_last_error()
 
 
+def test_shared_query_summary_checked():
+    p = P()
+    st = H.lib.hils_chunk_summary_shared_query(ctypes.byref(p), FAKE, FAKE, 2, 5, FAKE, FAKE, None)
+    assert st == 1 and b"hils_chunk_summary_shared_query: chunk range" in H.lib.hils_last_error()
+    st = H.lib.hils_chunk_summary_shared_query(ctypes.byref(p), FAKE, None, 0, 4, FAKE, FAKE, None)
+    assert st == 1 and b"q_shared" in H.lib.hils_last_error()
+    assert H.lib.hils_chunk_summary_shared_query(ctypes.byref(p), None, None, 3, 3, None, None, None) == 0
+
+
 def test_select_too_many_chunks_for_one_cta():
     p = P(T=1, L=1 << 20, q_pos0=(1 << 20) - 1)
     st = H.lib.hils_select_topk(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, None, 0, None)

@@ -148,3 +148,28 @@ def test_prefill_full_size_sampled():
     valid = idx >= 0
     assert torch.all(idx < n[None, None, :, None]) and torch.all((idx[..., 1:] > idx[..., :-1]) | ~valid[..., 1:])
     assert torch.all(valid.sum(-1) == torch.clamp(n, max=w.topk)[None, None, :])
+
+
+@pytest.mark.parametrize("dtype,Hq,Hkv,d,S,L", [
+    ("bf16", 16, 4, 128, 64, 64 * 37 + 19),  # streamed tensor-core kernel, ragged tail token
+    ("bf16", 8, 1, 128, 64, 64 * 20),        # G = 8
+    ("fp32", 4, 2, 64, 32, 32 * 9 + 5),      # CUDA-core kernel
+])
+def test_chunk_summary_shared_query(dtype, Hq, Hkv, d, S, L):
+    """Shared landmark query (one q' per head, Sec. 4) against the oracle, every element, plus a chunk
+    range that leaves the other chunks untouched."""
+    g = torch.Generator().manual_seed(77)
+    B = 2
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    k = torch.randn((B, Hkv, L, d), generator=g).to(dt)
+    qs = torch.randn((Hq, d), generator=g).to(dt)
+    geo = Geometry(B=B, T=1, L=L, Hq=Hq, Hkv=Hkv, d=d, S=S, topk=1, W=1)
+    ref_k, ref_b = oracle.chunk_summary_shared_query(geo, np64(k), np64(qs))
+    ks, bs = H.chunk_summary_shared_query(k.cuda(), qs.cuda(), S)
+    assert_close(ks, ref_k, TOL[dtype], "k_sum")
+    assert_close(bs, ref_b, BSUM_TOL, "b_sum")
+    ks2 = torch.full_like(ks, 7.0)
+    bs2 = torch.full_like(bs, 7.0)
+    H.chunk_summary_shared_query(k.cuda(), qs.cuda(), S, c_begin=3, c_end=7, k_sum=ks2, b_sum=bs2)
+    assert torch.equal(ks2[:, :, 3:7], ks[:, :, 3:7]) and torch.equal(bs2[:, :, 3:7], bs[:, :, 3:7])
+    assert bool((ks2[:, :, :3] == 7).all()) and bool((bs2[:, :, 7:] == 7).all())

@@ -106,6 +106,31 @@ def test_summary_chunk_range():
     assert np.all(part_k[:, :, :2] == 0) and np.all(part_k[:, :, 5:] == 0)
 
 
+def test_summary_shared_query_dominant_tokens():
+    """Shared landmark query (Sec. 4): q'[h] = 40 e_h serves every chunk of every sequence. Chunk c of KV
+    head g holds 40 e_h at token (c + h) mod S for each query head h of the group, so head h's summary of
+    chunk c is that token's key with b' ~ 0 (catches a wrong head, chunk or batch index into q')."""
+    g = Geometry(B=2, T=1, L=40, Hq=4, Hkv=2, d=8, S=8, topk=1, W=1)
+    r = rng(12)
+    k = r.standard_normal((2, 2, 40, 8)) * 0.5
+    for b in range(2):
+        for c in range(g.Nc):
+            for h in range(4):
+                k[b, h // 2, c * 8 + (c + h) % 8] = 0.0
+                k[b, h // 2, c * 8 + (c + h) % 8, h] = 40.0
+    qs = 40.0 * np.eye(8)[:4]
+    ks, bs = oracle.chunk_summary_shared_query(g, k, qs)
+    for b in range(2):
+        for h in range(4):
+            for c in range(g.Nc):
+                np.testing.assert_allclose(ks[b, h, c], k[b, h // 2, c * 8 + (c + h) % 8], atol=1e-12)
+                assert bs[b, h, c] < 1e-12
+    # and with q' = 0 the shared form is the uniform (mean-key, log S) summary
+    ks0, bs0 = oracle.chunk_summary_shared_query(g, k, np.zeros((4, 8)))
+    np.testing.assert_allclose(ks0[1, 3], k[1, 1].reshape(5, 8, 8).mean(axis=1), atol=1e-14)
+    np.testing.assert_allclose(bs0, math.log(8), atol=1e-14)
+
+
 def test_eq7_tangency_and_lower_bound():
     """Prop. 3.1 / Eq. 7: s^ = q^.k'/sqrt(d) + b' is the tangent of the chunk LogSumExp at q^ = q'_c, so it
     equals LSE_j(q'.k_j/sqrt(d)) there, and (LSE is convex) never exceeds LSE_j(q^.k_j/sqrt(d))."""
