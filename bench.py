@@ -395,6 +395,33 @@ def bench_decode(args, dist, dev, H, peaks, w: W.Workload, steps: int):
             "launches_per_step": 4}
 
 
+def bench_bsa(args, dist, dev, H, peaks):
+    """Naive BSA selection (exact chunk masses over every pre-window token + the group top-k) at the
+    prefill workload: the reference the HiLS selection approximates. Algorithmic flops: 2 d per (row,
+    head, candidate token)."""
+    w = W.PREFILL_BF16
+    x = W.prefill_inputs(w, seed=rank_seed(1000, dist.rank), device=dev)
+    idx = torch.empty((w.B, w.Hkv, w.T, w.topk), dtype=torch.int32, device=dev)
+    mass = torch.empty((w.B, w.Hq, w.T, w.Nc), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(mark):
+        H.bsa_select_topk(x["q"], x["k"], S=w.S, topk=w.topk, window=w.W, idx=idx, mass=mass)
+        mark()
+
+    steps = max(1, min(args.steps, 10))
+    _, total_ms, _ = timed_steps(steps, step, 3, flush, dist)
+    ms = dist.max(total_ms / steps)
+    cand_tokens = sum(window_left(p, w.W, w.S) for p in range(w.T)) * w.B * w.Hq
+    flops = 2 * w.d * cand_tokens
+    tf = flops / (ms / 1e3) / 1e12
+    return {"workload": w.name, "ms": ms, "flops": flops,
+            "roofline": {"bound": "tensor", "kernel": "hils_bsa_select_topk (masses + top-k)", "achieved": tf,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"],
+                         "traffic": None},
+            "launches_per_step": 2}
+
+
 def bench_train(args, dist, dev, H, peaks):
     w = W.TRAIN_BF16
     x = W.prefill_inputs(w, seed=rank_seed(3000, dist.rank), device=dev, with_dout=True)
@@ -538,6 +565,9 @@ def profile_case(args):
         if st == "select":
             fn = lambda: H.select_topk(x["q_hat"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S, topk=w.topk, window=w.W,
                                        idx=idx)
+        elif st == "bsa":
+            mass = torch.empty((w.B, w.Hq, w.T, w.Nc), dtype=torch.float32, device=dev)
+            fn = lambda: H.bsa_select_topk(x["q"], x["k"], S=w.S, topk=w.topk, window=w.W, idx=idx, mass=mass)
         elif st == "attn":
             fn = lambda: H.attn_fwd(x["q"], x["k"], x["v"], x["q_hat"], k_sum, b_sum, idx, S=w.S, window=w.W,
                                     out=out, lse=lse)
@@ -560,7 +590,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="hils", choices=("hils", "reference"))
     ap.add_argument("--quick", action="store_true", help="headline only (no decode sweep / training blocks)")
-    ap.add_argument("--profile", choices=("summary", "select", "attn", "decode", "bwd"),
+    ap.add_argument("--profile", choices=("summary", "select", "attn", "decode", "bwd", "bsa"),
                     help="run --steps untimed launches of one stage for an ncu capture; no bench line")
     args = ap.parse_args()
     if args.profile:
@@ -596,6 +626,7 @@ def main():
                                      q_pos0=W.DECODE_BF16.L - 4)
             extra["decode_multi"] = bench_decode(args, dist, dev, H, peaks, wm, 64)
             extra["train"] = bench_train(args, dist, dev, H, peaks)
+            extra["bsa_select"] = bench_bsa(args, dist, dev, H, peaks)
         cpu = None
         if dist.world == 1:
             cpu = cpu_baseline(pre["x"], w)

@@ -30,6 +30,10 @@ cudaError_t launch_select_tc(const Dims &D, const void *q_hat, const void *k_sum
 unsigned int select_tc_error_flags(bool clear);
 unsigned int summary_error_flags(bool clear);
 unsigned int attn_bwd_tc_error_flags(bool clear);
+unsigned int bsa_error_flags(bool clear);
+int bsa_max_candidates(const Dims &D);
+cudaError_t launch_bsa_select_topk(const Dims &D, int dtype, const void *q, const void *k, int *idx, float *gap,
+                                   float *mass, cudaStream_t stream);
 
 namespace {
 
@@ -111,6 +115,9 @@ hils_status check_device_errors() {
     if (attn_bwd_tc_error_flags(true) != 0)
         return fail(HILS_ERR_TIMEOUT, "hils_check: a tensor-core backward tile's wait expired; that call's "
                     "gradients are invalid");
+    if (bsa_error_flags(true) != 0)
+        return fail(HILS_ERR_TIMEOUT, "hils_check: a naive-BSA mass tile's wait expired; that call's masses and ids "
+                    "are invalid");
     if (decode_error_flags(true) != 0)
         return fail(HILS_ERR_TIMEOUT, "hils_check: a decode tile's bulk copy did not complete within its wait "
                     "budget; that call's output is invalid");
@@ -211,6 +218,23 @@ hils_status hils_select_topk(const hils_params *p, const void *q_hat, const void
     if (select_tc_supported(D, p->dtype))
         return cuda_status(launch_select_tc(D, q_hat, k_sum, b_sum, idx, gap, (cudaStream_t)stream), fn);
     return cuda_status(launch_select_topk(D, p->dtype, q_hat, k_sum, b_sum, idx, gap, (cudaStream_t)stream), fn);
+}
+
+hils_status hils_bsa_select_topk(const hils_params *p, const void *q, const void *k, int32_t *idx, float *gap,
+                                 float *mass, hils_stream_t stream) {
+    const char *fn = "hils_bsa_select_topk";
+    Dims D;
+    hils_status st = resolve(p, fn, &D);
+    if (st != HILS_OK) return st;
+    if (D.topk > 32) return fail(HILS_ERR_UNSUPPORTED, "%s: topk %d > 32", fn, D.topk);
+    if (bsa_max_candidates(D) > 1024)
+        return fail(HILS_ERR_UNSUPPORTED, "%s: %d candidate chunks per row > 1024", fn, bsa_max_candidates(D));
+    HILS_REQUIRE_PTR(q);
+    HILS_REQUIRE_PTR(k);
+    HILS_REQUIRE_PTR(idx);
+    if (D.Nc > 0) HILS_REQUIRE_PTR(mass);
+    if (gap != nullptr && !aligned16(gap)) return fail(HILS_ERR_INVALID_ARG, "%s: gap is not 16-byte aligned", fn);
+    return cuda_status(launch_bsa_select_topk(D, p->dtype, q, k, idx, gap, mass, (cudaStream_t)stream), fn);
 }
 
 hils_status hils_attn_fwd(const hils_params *p, const void *q, const void *k, const void *v, const void *q_hat,

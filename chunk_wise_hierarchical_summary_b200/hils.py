@@ -27,7 +27,7 @@ OP_SUMMARY, OP_SELECT, OP_ATTN_FWD, OP_DECODE, OP_ATTN_BWD = 0, 1, 2, 3, 4
 
 # Every symbol include/hils.h declares (checked by the tests against the header and the library).
 EXPORTED = ("hils_workspace_size", "hils_chunk_summary", "hils_chunk_summary_shared_query", "hils_select_topk",
-            "hils_attn_fwd", "hils_decode", "hils_attn_bwd", "hils_check", "hils_status_string", "hils_last_error",
+            "hils_bsa_select_topk", "hils_attn_fwd", "hils_decode", "hils_attn_bwd", "hils_check", "hils_status_string", "hils_last_error",
             "hils_version", "hils_decode_noalloc")
 
 
@@ -56,6 +56,8 @@ def _load() -> ctypes.CDLL:
     lib.hils_chunk_summary_shared_query.restype = st
     lib.hils_select_topk.argtypes = [P, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.hils_select_topk.restype = st
+    lib.hils_bsa_select_topk.argtypes = [P, vp, vp, vp, vp, vp, vp]
+    lib.hils_bsa_select_topk.restype = st
     lib.hils_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.hils_attn_fwd.restype = st
     lib.hils_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
@@ -192,6 +194,32 @@ def select_topk(q_hat, k_sum, b_sum, *, Hkv: int, L: int, S: int, topk: int, win
     _raise(lib.hils_select_topk(ctypes.byref(p), _ptr(q_hat), _ptr(k_sum), _ptr(b_sum), _ptr(idx), _ptr(gap),
                                 _ptr(ws), nws, _stream(dev)))
     return (idx, gap) if gap is not None else idx
+
+
+def bsa_select_topk(q, k, *, S: int, topk: int, window: int, q_pos0: int = 0, scale: float = 0.0,
+                    with_gap: bool = False, idx=None, gap=None, mass=None):
+    """Naive BSA selection (Sec. 2): exact chunk log-masses and the GQA top-k on them. q [B,Hq,T,d],
+    k [B,Hkv,L,d] -> (idx [B,Hkv,T,topk] int32, gap [B,Hkv,T] fp32 or None, mass [B,Hq,T,Nc] fp32; entries
+    of mass at c >= n_i are not written)."""
+    B, Hq, T, d = q.shape
+    Hkv, L = k.shape[1], k.shape[2]
+    dev, dt = q.device, q.dtype
+    Nc = L // S
+    _check("k", k, dt, (B, Hkv, L, d), dev)
+    if idx is None:
+        idx = torch.empty((B, Hkv, T, topk), dtype=torch.int32, device=dev)
+    _check("idx", idx, torch.int32, (B, Hkv, T, topk), dev)
+    if with_gap and gap is None:
+        gap = torch.empty((B, Hkv, T), dtype=torch.float32, device=dev)
+    if gap is not None:
+        _check("gap", gap, torch.float32, (B, Hkv, T), dev)
+    if mass is None:
+        mass = torch.empty((B, Hq, T, Nc), dtype=torch.float32, device=dev)
+    _check("mass", mass, torch.float32, (B, Hq, T, Nc), dev)
+    p = make_params(B, T, L, Hq, Hkv, d, S, topk, window, q_pos0, scale, dt)
+    _raise(lib.hils_bsa_select_topk(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(idx), _ptr(gap), _ptr(mass),
+                                    _stream(dev)))
+    return idx, gap, mass
 
 
 def attn_fwd(q, k, v, q_hat, k_sum, b_sum, idx, *, S: int, window: int, q_pos0: int = 0, scale: float = 0.0,

@@ -121,6 +121,22 @@ HILS_API hils_status hils_select_topk(const hils_params *p, const void *q_hat, c
                              hils_stream_t stream);
 
 /*
+ * Naive block-sparse attention selection (Sec. 2), the exact counterpart of hils_select_topk: for every
+ * (b, query head h, row i) at position p with n = n_p candidates, the exact chunk mass
+ *   mass[b,h,i,c] = LSE_{j in chunk c} tau q[b,h,i].k[b,h/G,j]   for c < n (entries c >= n untouched),
+ * then the group rule of hils_select_topk with mass in place of s^: per-head normalisation over the
+ * candidates, max over the group's heads, the min(topk, n) largest by (score desc, c asc).
+ * idx [B, Hkv, T, topk] int32 (ascending ids, -1 padded); gap (nullable) [B, Hkv, T] as in
+ * hils_select_topk; mass [B, Hq, T, Nc] fp32 (nullable when Nc = 0). q [B, Hq, T, d], k [B, Hkv, L, d].
+ * Reads every pre-window key once per query row (O(T * L) work): a reference for selection quality,
+ * not a step of the HiLS path. Needs topk <= 32 and at most 1024 candidates per row
+ * (HILS_ERR_UNSUPPORTED otherwise). Tensor cores for bf16, d 128, S 64, G in {1, 2, 4, 8}.
+ * No workspace.
+ */
+HILS_API hils_status hils_bsa_select_topk(const hils_params *p, const void *q, const void *k, int32_t *idx, float *gap,
+                                          float *mass, hils_stream_t stream);
+
+/*
  * Stages (c)+(d), Eq. 10 (chunked prefill form): for every (b, h, row i) at position p:
  *   window logits s_j = tau q.k_j, j in [l_p, p];  for each selected chunk c (idx, as a set):
  *   s^_c (as above), L_c = LSE_{j in c} s_j, o_c = sum_j exp(s_j - L_c) v_j;

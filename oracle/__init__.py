@@ -7,6 +7,7 @@ Every function converts its inputs to contiguous fp64 (int32 for idx) and calls 
 statement in hils_oracle.c, which cites the paper section / equation each step follows:
   chunk_summary  Eq. 8 (Prop. 3.1)            select_topk  Sec. 3 RQ1 + Sec. 4 GQA selection
   chunk_summary_shared_query  Eq. 8 with one landmark query per head (Sec. 4)
+  bsa_select_topk  naive BSA (Sec. 2): exact chunk masses, same group top-k
   attn_fwd       Eq. 10, chunked form          eq10_tokenwise  Eq. 10, token by token
   attn_bwd       gradients of the above with the selection held fixed
   decode         select_topk + attn_fwd for one query at position L-1
@@ -84,6 +85,7 @@ def _load():
         lib.orc_window.argtypes = [P, I, I]
         lib.orc_chunk_summary.argtypes = [P, D, D, ctypes.c_int, ctypes.c_int, D, D]
         lib.orc_select_topk.argtypes = [P, D, D, D, I, D]
+        lib.orc_bsa_select_topk.argtypes = [P, D, D, I, D, D]
         lib.orc_attn_fwd.argtypes = [P, D, D, D, D, D, D, I, D, D]
         lib.orc_eq10_tokenwise.argtypes = [P, D, D, D, D, D, D, I, D, D]
         lib.orc_attn_bwd.argtypes = [P, D, D, D, D, D, I, D, D, D, D, D, D]
@@ -157,6 +159,19 @@ def select_topk(g: Geometry, q_hat, k_sum, b_sum):
     gap = np.zeros((g.B, g.Hkv, g.T))
     _load().orc_select_topk(ctypes.byref(g._c()), _pd(qh), _pd(ks), _pd(bs), _pi(idx), _pd(gap))
     return idx, gap
+
+
+def bsa_select_topk(g: Geometry, q, k):
+    """Naive BSA (Sec. 2): exact log chunk masses M [B,Hq,T,Nc] (LSE over the chunk's token logits, for
+    the row's candidates; NaN elsewhere) and the group top-k on them (same rule as select_topk), with
+    its gap. Returns (idx, gap, mass)."""
+    qq = _f64(q, (g.B, g.Hq, g.T, g.d))
+    kk = _f64(k, (g.B, g.Hkv, g.L, g.d))
+    idx = np.zeros((g.B, g.Hkv, g.T, g.topk), np.int32)
+    gap = np.zeros((g.B, g.Hkv, g.T))
+    mass = np.full((g.B, g.Hq, g.T, g.Nc), np.nan)
+    _load().orc_bsa_select_topk(ctypes.byref(g._c()), _pd(qq), _pd(kk), _pi(idx), _pd(gap), _pd(mass))
+    return idx, gap, mass
 
 
 def attn_fwd(g: Geometry, q, k, v, q_hat, k_sum, b_sum, idx):

@@ -152,12 +152,38 @@ static int int_cmp(const void *x, const void *y) {
 }
 
 /*
- * Sec. 3 RQ1 (top-k over the retrieval scores) with Sec. 4 "GQA": for every (b, KV group g, row i)
- * at position pos with n candidates:
- *   s^_{h,c} for c < n and every head h of the group; per-head log-normalised weight
- *   s^_{h,c} - LSE_{c'<n} s^_{h,c'}; group score g_c = max over the group's heads;
+ * Sec. 4 "GQA" selection from per-head chunk scores sc[hh*n + c] (hh < G, c < n) of one (b, g, row):
+ *   per-head log-normalised weight sc_{h,c} - LSE_{c'<n} sc_{h,c'}; group score g_c = max over heads;
  *   keep min(topk, n) candidates by (g desc, c asc); write them ascending, pad with -1.
  * gap (nullable) = g_(topk) - g_(topk+1) in the sorted order, +inf when n <= topk.
+ */
+static void group_topk(int G, int n, int K, const double *sc, int *out, double *gp) {
+    for (int t = 0; t < K; ++t) out[t] = -1;
+    if (n == 0) {
+        if (gp) *gp = INFINITY;
+        return;
+    }
+    cand_t *cand = (cand_t *)malloc(sizeof(cand_t) * n);
+    for (int c = 0; c < n; ++c) { cand[c].g = -INFINITY; cand[c].c = c; }
+    for (int hh = 0; hh < G; ++hh) {
+        const double z = logsumexp(sc + (size_t)hh * n, n);
+        for (int c = 0; c < n; ++c) {
+            double w = sc[(size_t)hh * n + c] - z;
+            if (w > cand[c].g) cand[c].g = w;
+        }
+    }
+    qsort(cand, n, sizeof(cand_t), cand_cmp);
+    const int kk = n < K ? n : K;
+    for (int t = 0; t < kk; ++t) out[t] = cand[t].c;
+    qsort(out, kk, sizeof(int), int_cmp);
+    if (gp) *gp = (n > K) ? cand[K - 1].g - cand[K].g : INFINITY;
+    free(cand);
+}
+
+/*
+ * Sec. 3 RQ1 (top-k over the retrieval scores) with Sec. 4 "GQA": for every (b, KV group g, row i)
+ * at position pos with n candidates, s^_{h,c} for c < n and every head h of the group, then the
+ * group selection above.
  * Pinned by: planted dominant chunks, tie rule on identical chunks, per-head shift invariance,
  * G = 1 reduction (top-k of raw s^), and the naive-BSA special case.
  */
@@ -171,32 +197,54 @@ void orc_select_topk(const orc_params *p, const double *q_hat, const double *k_s
                 const int pos = p->q_pos0 + i;
                 const int n = window_left(p, pos) / p->S;
                 int *out = idx + (((size_t)b * p->Hkv + g) * p->T + i) * K;
-                for (int t = 0; t < K; ++t) out[t] = -1;
                 double *gp = gap ? gap + ((size_t)b * p->Hkv + g) * p->T + i : NULL;
-                if (n == 0) {
-                    if (gp) *gp = INFINITY;
-                    continue;
-                }
-                cand_t *cand = (cand_t *)malloc(sizeof(cand_t) * n);
-                double *sh = (double *)malloc(sizeof(double) * n);
-                for (int c = 0; c < n; ++c) { cand[c].g = -INFINITY; cand[c].c = c; }
+                double *sh = (double *)malloc(sizeof(double) * ((size_t)G * n + 1));
                 for (int hh = 0; hh < G; ++hh) {
                     const int h = g * G + hh;
                     const double *qh = q_hat + (((size_t)b * p->Hq + h) * p->T + i) * p->d;
-                    for (int c = 0; c < n; ++c) sh[c] = retrieval_score(p, qh, k_sum, b_sum, b, h, c);
-                    const double z = logsumexp(sh, n);
+                    for (int c = 0; c < n; ++c) sh[(size_t)hh * n + c] = retrieval_score(p, qh, k_sum, b_sum, b, h, c);
+                }
+                group_topk(G, n, K, sh, out, gp);
+                free(sh);
+            }
+}
+
+/*
+ * Naive BSA (Sec. 2): the exact chunk mass of candidate c for row i under head h is
+ * sum_{j in c} exp(s_ij), s_ij = tau q_i.k_j; its log, M_{h,c} = LSE_{j in c} s_ij, takes the place of
+ * s^ in the same group selection (per-head normalisation over the candidates, max over the group's
+ * heads, top-k by (score desc, id asc)). mass (nullable) [B,Hq,T,Nc]: M_{h,c} for c < n, entries
+ * c >= n left untouched. With G = 1 this is top-k by raw chunk mass, the rule Sec. 2 states.
+ * Pinned by: brute-force chunk masses and top-k on tiny inputs, equality with the HiLS selection on
+ * chunk-constant keys (where the summary is exact, Prop. 3.1), and a planted two-head GQA case.
+ */
+void orc_bsa_select_topk(const orc_params *p, const double *q, const double *k, int *idx, double *gap,
+                         double *mass) {
+    const int G = p->Hq / p->Hkv, K = p->topk, S = p->S, d = p->d, Nc = p->L / p->S;
+    const double tau = tau_of(p);
+#pragma omp parallel for collapse(3) schedule(dynamic)
+    for (int b = 0; b < p->B; ++b)
+        for (int g = 0; g < p->Hkv; ++g)
+            for (int i = 0; i < p->T; ++i) {
+                const int pos = p->q_pos0 + i;
+                const int n = window_left(p, pos) / S;
+                int *out = idx + (((size_t)b * p->Hkv + g) * p->T + i) * K;
+                double *gp = gap ? gap + ((size_t)b * p->Hkv + g) * p->T + i : NULL;
+                double *m = (double *)malloc(sizeof(double) * ((size_t)G * n + 1));
+                double *s = (double *)malloc(sizeof(double) * S);
+                for (int hh = 0; hh < G; ++hh) {
+                    const int h = g * G + hh;
+                    const double *qi = q + (((size_t)b * p->Hq + h) * p->T + i) * d;
                     for (int c = 0; c < n; ++c) {
-                        double w = sh[c] - z;
-                        if (w > cand[c].g) cand[c].g = w;
+                        for (int j = 0; j < S; ++j)
+                            s[j] = tau * dot(qi, k + (((size_t)b * p->Hkv + g) * p->L + (size_t)c * S + j) * d, d);
+                        m[(size_t)hh * n + c] = logsumexp(s, S);
+                        if (mass) mass[(((size_t)b * p->Hq + h) * p->T + i) * Nc + c] = m[(size_t)hh * n + c];
                     }
                 }
-                qsort(cand, n, sizeof(cand_t), cand_cmp);
-                const int kk = n < K ? n : K;
-                for (int t = 0; t < kk; ++t) out[t] = cand[t].c;
-                qsort(out, kk, sizeof(int), int_cmp);
-                if (gp) *gp = (n > K) ? cand[K - 1].g - cand[K].g : INFINITY;
-                free(cand);
-                free(sh);
+                group_topk(G, n, K, m, out, gp);
+                free(s);
+                free(m);
             }
 }
 

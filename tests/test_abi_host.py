@@ -124,6 +124,20 @@ def test_shared_query_summary_checked():
     assert H.lib.hils_chunk_summary_shared_query(ctypes.byref(p), None, None, 3, 3, None, None, None) == 0
 
 
+def test_bsa_select_rules():
+    p = P(topk=33)
+    st = H.lib.hils_bsa_select_topk(ctypes.byref(p), FAKE, FAKE, FAKE, None, FAKE, None)
+    assert st == 2 and b"topk 33 > 32" in H.lib.hils_last_error()
+    p = P(T=1, L=1 << 20, q_pos0=(1 << 20) - 1)
+    st = H.lib.hils_bsa_select_topk(ctypes.byref(p), FAKE, FAKE, FAKE, None, FAKE, None)
+    assert st == 2 and b"> 1024" in H.lib.hils_last_error()
+    p = P()
+    st = H.lib.hils_bsa_select_topk(ctypes.byref(p), FAKE, FAKE, FAKE, None, None, None)
+    assert st == 1 and b"mass is NULL" in H.lib.hils_last_error()
+    st = H.lib.hils_bsa_select_topk(ctypes.byref(p), FAKE, FAKE, FAKE, ctypes.c_void_p(FAKE.value + 4), FAKE, None)
+    assert st == 1 and b"gap is not 16-byte aligned" in H.lib.hils_last_error()
+
+
 def test_select_too_many_chunks_for_one_cta():
     p = P(T=1, L=1 << 20, q_pos0=(1 << 20) - 1)
     st = H.lib.hils_select_topk(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, None, 0, None)

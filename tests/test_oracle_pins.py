@@ -267,6 +267,65 @@ def test_select_head_group_mapping():
         np.testing.assert_array_equal(idx[:, grp:grp + 1], i1)
 
 
+# ---------------------------------------------------------------- naive BSA (Sec. 2)
+
+def test_bsa_masses_brute_force_and_mha_topk():
+    """Naive BSA on a tiny MHA case: every chunk mass equals the direct sum of exp(tau q.k_j) over the chunk's
+    tokens, and the selection is the top-k of those sums by (mass desc, id asc), as Sec. 2 states."""
+    g = Geometry(B=2, T=40, L=40, Hq=2, Hkv=2, d=4, S=4, topk=3, W=6, scale=0.7)
+    r = rng(31)
+    q = r.standard_normal((2, 2, 40, 4))
+    k = r.standard_normal((2, 2, 40, 4))
+    idx, gap, mass = oracle.bsa_select_topk(g, q, k)
+    for b in range(2):
+        for h in range(2):
+            for i in range(40):
+                left = max(0, i - 6 + 1) // 4 * 4
+                n = left // 4
+                sums = [sum(math.exp(0.7 * float(q[b, h, i] @ k[b, h, j])) for j in range(4 * c, 4 * c + 4))
+                        for c in range(n)]
+                np.testing.assert_allclose(np.exp(mass[b, h, i, :n]), sums, rtol=1e-12)
+                assert np.all(np.isnan(mass[b, h, i, n:]))
+                order = sorted(range(n), key=lambda c: (-sums[c], c))[:3]
+                expect = sorted(order) + [-1] * (3 - len(order))
+                assert idx[b, h, i].tolist() == expect, (b, h, i)
+
+
+def test_bsa_masses_partition_the_pre_window_logits():
+    """The candidate chunks tile the tokens left of the window: LSE over the chunk masses equals the LSE of
+    every logit s_ij with j < l_p (catches a chunk boundary or a token dropped or counted twice)."""
+    g = Geometry(B=1, T=200, L=200, Hq=4, Hkv=2, d=8, S=16, topk=4, W=40)
+    x = rand_problem(g, seed=32)
+    _, _, mass = oracle.bsa_select_topk(g, x["q"], x["k"])
+    left, n = oracle.window(g)
+    for h in range(4):
+        for i in range(0, 200, 7):
+            if n[i] == 0:
+                continue
+            s = g.tau() * x["k"][0, h // 2, :left[i]] @ x["q"][0, h, i]
+            assert abs(logsumexp(mass[0, h, i, :n[i]]) - logsumexp(s)) < 1e-11
+
+
+def test_bsa_equals_hils_on_chunk_constant_keys():
+    """With every key of a chunk equal, the landmark summary is exact (k' = k_c, b' = log S, Prop. 3.1), so
+    the HiLS selection with q^ = q is the naive BSA selection and s^ is the exact log mass."""
+    g = Geometry(B=1, T=160, L=160, Hq=4, Hkv=2, d=8, S=8, topk=3, W=24)
+    r = rng(33)
+    kc = r.standard_normal((1, 2, g.Nc, 8))
+    k = np.repeat(kc, 8, axis=2)
+    q = r.standard_normal((1, 4, 160, 8))
+    idx_b, gap_b, mass = oracle.bsa_select_topk(g, q, k)
+    ks, bs = oracle.chunk_summary(g, k, r.standard_normal((1, 4, g.Nc, 8)))
+    idx_h, gap_h = oracle.select_topk(g, q, ks, bs)
+    np.testing.assert_array_equal(idx_b, idx_h)
+    np.testing.assert_allclose(gap_b, gap_h, rtol=1e-9, atol=1e-12)
+    left, n = oracle.window(g)
+    for h in range(4):
+        for i in range(0, 160, 5):
+            closed = g.tau() * kc[0, h // 2, :n[i]] @ q[0, h, i] + math.log(8)
+            np.testing.assert_allclose(mass[0, h, i, :n[i]], closed, rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------- Eq. 10 attention
 
 def test_eq10_golden_three_tokens():
