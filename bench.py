@@ -422,6 +422,28 @@ def bench_bsa(args, dist, dev, H, peaks):
             "launches_per_step": 2}
 
 
+def bench_select_qcal(args, dist, dev, H):
+    """Selection with Q-Cal fused (q^ formed from q in shared memory) against the plain selection on a
+    precomputed q^, both at the prefill workload on the same summaries."""
+    w = W.PREFILL_BF16
+    x = W.prefill_inputs(w, seed=rank_seed(1000, dist.rank), device=dev)
+    k_sum, b_sum = H.chunk_summary(x["k"], x["q_land"], w.S)
+    idx = torch.empty((w.B, w.Hkv, w.T, w.topk), dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(mark):
+        H.select_topk_qcal(x["q"], x["w_down"], x["w_up"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S, topk=w.topk,
+                           window=w.W, idx=idx)
+        mark()
+        H.select_topk(x["q_hat"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S, topk=w.topk, window=w.W, idx=idx)
+        mark()
+
+    steps = max(1, min(args.steps, 10))
+    stage_ms, _, _ = timed_steps(steps, step, 3, flush, dist)
+    return {"workload": w.name, "fused_ms": dist.max(stage_ms[0] / steps), "unfused_ms": dist.max(stage_ms[1] / steps),
+            "note": "fused: hils_select_topk_qcal from q, W_down, W_up; unfused: hils_select_topk from q^"}
+
+
 def bench_train(args, dist, dev, H, peaks):
     w = W.TRAIN_BF16
     x = W.prefill_inputs(w, seed=rank_seed(3000, dist.rank), device=dev, with_dout=True)
@@ -627,6 +649,7 @@ def main():
             extra["decode_multi"] = bench_decode(args, dist, dev, H, peaks, wm, 64)
             extra["train"] = bench_train(args, dist, dev, H, peaks)
             extra["bsa_select"] = bench_bsa(args, dist, dev, H, peaks)
+            extra["select_qcal"] = bench_select_qcal(args, dist, dev, H)
         cpu = None
         if dist.world == 1:
             cpu = cpu_baseline(pre["x"], w)

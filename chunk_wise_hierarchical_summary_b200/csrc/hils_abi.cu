@@ -31,6 +31,8 @@ unsigned int select_tc_error_flags(bool clear);
 unsigned int summary_error_flags(bool clear);
 unsigned int attn_bwd_tc_error_flags(bool clear);
 unsigned int bsa_error_flags(bool clear);
+cudaError_t launch_select_tc_qcal(const Dims &D, const void *q, const void *w_down, const void *w_up,
+                                  const void *k_sum, const float *b_sum, int *idx, float *gap, cudaStream_t stream);
 int bsa_max_candidates(const Dims &D);
 cudaError_t launch_bsa_select_topk(const Dims &D, int dtype, const void *q, const void *k, int *idx, float *gap,
                                    float *mass, cudaStream_t stream);
@@ -218,6 +220,27 @@ hils_status hils_select_topk(const hils_params *p, const void *q_hat, const void
     if (select_tc_supported(D, p->dtype))
         return cuda_status(launch_select_tc(D, q_hat, k_sum, b_sum, idx, gap, (cudaStream_t)stream), fn);
     return cuda_status(launch_select_topk(D, p->dtype, q_hat, k_sum, b_sum, idx, gap, (cudaStream_t)stream), fn);
+}
+
+hils_status hils_select_topk_qcal(const hils_params *p, const void *q, const void *w_down, const void *w_up,
+                                  int32_t rank, const void *k_sum, const float *b_sum, int32_t *idx, float *gap,
+                                  hils_stream_t stream) {
+    const char *fn = "hils_select_topk_qcal";
+    Dims D;
+    hils_status st = resolve(p, fn, &D);
+    if (st != HILS_OK) return st;
+    if (rank != 32) return fail(HILS_ERR_UNSUPPORTED, "%s: rank %d (the fused path takes 32)", fn, rank);
+    if (!select_tc_supported(D, p->dtype))
+        return fail(HILS_ERR_UNSUPPORTED, "%s: needs bf16, d 128, G <= 4, topk <= 32 and 1..128 candidates per row "
+                    "(otherwise form q^ and call hils_select_topk)", fn);
+    HILS_REQUIRE_PTR(q);
+    HILS_REQUIRE_PTR(w_down);
+    HILS_REQUIRE_PTR(w_up);
+    HILS_REQUIRE_PTR(k_sum);
+    HILS_REQUIRE_PTR(b_sum);
+    HILS_REQUIRE_PTR(idx);
+    if (gap != nullptr && !aligned16(gap)) return fail(HILS_ERR_INVALID_ARG, "%s: gap is not 16-byte aligned", fn);
+    return cuda_status(launch_select_tc_qcal(D, q, w_down, w_up, k_sum, b_sum, idx, gap, (cudaStream_t)stream), fn);
 }
 
 hils_status hils_bsa_select_topk(const hils_params *p, const void *q, const void *k, int32_t *idx, float *gap,

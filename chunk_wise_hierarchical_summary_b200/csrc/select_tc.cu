@@ -10,7 +10,13 @@
 //            (score desc, chunk id asc); each thread keeps its block's best K1 in a sorted register list.
 //   phase 3  one thread per row merges the four lists: top-k ids (ascending) and the gap.
 // Rows whose candidates exceed 128 chunks use the general kernel (select.cu).
+//
+// Fused Q-Cal (Sec. 4, q^ = q + W_up W_down h with h = q and one rank-32 pair for all heads): the
+// loaded tile holds q instead of q^; warps 8-15 (16 rows each) rewrite it in place as q^ before the
+// head's MMA: z = W_down q (mma.sync, N = 32), then q + W_up z with z split into bf16 hi + lo, rounded
+// once to bf16 into the swizzled tile. The q^ tensor is never formed in HBM.
 #include "internal.h"
+#include "mma_sync.cuh"
 #include "tcgen05.cuh"
 
 namespace hils {
@@ -23,16 +29,82 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kRows = 128;
 constexpr int kStageBytes = 65536;  // q^ tile (32 KiB) + k' tile (32 KiB)
+constexpr int kRank = 32;           // Q-Cal rank of the fused path
+constexpr int kWdRow = 272;         // W_down row (128 bf16) padded: conflict-free fragment loads
+constexpr int kWuRow = 80;          // W_up row (32 bf16) padded
+constexpr int kWdBytes = kRank * kWdRow;
+constexpr int kWuBytes = 128 * kWuRow;
+
+// q -> q^ = q + W_up (W_down q) for rows rb .. rb+15 of a 128 x 128 bf16 tile in the 128-byte-swizzled
+// K-major layout (two 64-column halves of 16 KiB), in place. One warp.
+__device__ __forceinline__ void qcal_rows(unsigned char *A, const unsigned char *wsm, int rb, int lane) {
+    const int g8 = lane >> 2, t4 = lane & 3, mi = lane >> 3, r8 = lane & 7;
+    const uint32_t Ab = smem_u32(A);
+    const unsigned char *wd = wsm, *wu = wsm + kWdBytes;
+    float z[4][4];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) z[nt][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+        const int row = rb + r8 + (mi & 1) * 8;
+        const int ch = (ks & 3) * 2 + (mi >> 1);
+        uint32_t a[4];
+        ldsm_x4(Ab + (ks >> 2) * 16384 + row * 128 + ((ch ^ (row & 7)) << 4), a);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            const unsigned char *p = wd + (nt * 8 + g8) * kWdRow + (ks * 16 + 2 * t4) * 2;
+            mma_16816(z[nt], a, ld_u32(p), ld_u32(p + 16));
+        }
+    }
+    __syncwarp();  // every lane's fragment loads of these rows are done before any lane rewrites them
+    // z (16 x 32, accumulator layout) is the A operand of the second product: k-step kk covers the
+    // accumulator tiles 2kk and 2kk+1. Split into bf16 hi + lo so z keeps ~16 significant bits.
+    uint32_t ah[2][4], al[2][4];
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float x = z[2 * kk + (e >> 1)][2 * (e & 1)], y = z[2 * kk + (e >> 1)][2 * (e & 1) + 1];
+            const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+            const float2 hf = __bfloat1622float2(h);
+            const __nv_bfloat162 l = __floats2bfloat162_rn(x - hf.x, y - hf.y);
+            ah[kk][e] = *reinterpret_cast<const uint32_t *>(&h);
+            al[kk][e] = *reinterpret_cast<const uint32_t *>(&l);
+        }
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+            const unsigned char *p = wu + (nt * 8 + g8) * kWuRow + (kk * 16 + 2 * t4) * 2;
+            const uint32_t b0 = ld_u32(p), b1 = ld_u32(p + 16);
+            mma_16816(c, ah[kk], b0, b1);
+            mma_16816(c, al[kk], b0, b1);
+        }
+        const int col = nt * 8 + 2 * t4;
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const int row = rb + g8 + 8 * hr;
+            unsigned char *qp = A + (col >> 6) * 16384 + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + (col & 7) * 2;
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(qp));
+            *reinterpret_cast<__nv_bfloat162 *>(qp) = __floats2bfloat162_rn(f.x + c[2 * hr], f.y + c[2 * hr + 1]);
+        }
+    }
+}
 
 __device__ unsigned int g_select_tc_errors = 0;
 
-template <int K1MAX, int GATHER>
+template <int K1MAX, int GATHER, int QCAL>
 __global__ void __launch_bounds__(kThreads, 1)
 select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, Dims D,
                  const float *__restrict__ b_sum, int *__restrict__ idx, float *__restrict__ gap,
-                 int *__restrict__ ws_idx, float *__restrict__ ws_shat) {
+                 int *__restrict__ ws_idx, float *__restrict__ ws_shat, const __nv_bfloat16 *__restrict__ w_down,
+                 const __nv_bfloat16 *__restrict__ w_up) {
     extern __shared__ unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t tma_bar[2], mma_bar[2], done_bar;
+    __shared__ __align__(8) uint64_t tma_bar[2], mma_bar[2], done_bar, qcal_bar[2];
+    __shared__ __align__(16) unsigned char wsm[QCAL ? kWdBytes + kWuBytes : 16];
     __shared__ uint32_t s_tmem;
     __shared__ float bs[4][kRows];
     __shared__ float lse[4][kRows];
@@ -46,10 +118,18 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
         tmem_alloc(&s_tmem, ncols);
         tmem_relinquish();
     }
+    if constexpr (QCAL != 0) {
+        // W_down [32][128] and W_up [128][32] (bf16, 8 KiB each) into padded rows: one 16-byte piece a thread
+        const uint4 wd = reinterpret_cast<const uint4 *>(w_down)[tid];
+        const uint4 wu = reinterpret_cast<const uint4 *>(w_up)[tid];
+        *reinterpret_cast<uint4 *>(wsm + (tid >> 4) * kWdRow + (tid & 15) * 16) = wd;
+        *reinterpret_cast<uint4 *>(wsm + kWdBytes + (tid >> 2) * kWuRow + (tid & 3) * 16) = wu;
+    }
     if (tid == 32) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tma_bar[i], 1);
             mbar_init(&mma_bar[i], 1);
+            mbar_init(&qcal_bar[i], 8);
         }
         mbar_init(&done_bar, 1);
         fence_mbar_init();
@@ -75,7 +155,8 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
             const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
             for (int hh = 0; hh < G && ok; ++hh) {
                 const int st = hh & 1;
-                if (!mbar_wait_bounded(&tma_bar[st], (hh >> 1) & 1)) { ok = false; break; }
+                // the tile is ready once TMA has landed it (and, with Q-Cal, warps 8-15 have rewritten it)
+                if (!mbar_wait_bounded(QCAL ? &qcal_bar[st] : &tma_bar[st], (hh >> 1) & 1)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t A = smem_u32(base + st * kStageBytes), Bt = A + 32768;
 #pragma unroll
@@ -94,6 +175,20 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
             umma_commit(&done_bar);  // arrives once every MMA issued above has completed
         }
         __syncwarp();
+    } else if (warp >= 8) {
+        if constexpr (QCAL != 0) {
+            for (int hh = 0; hh < G; ++hh) {
+                const int st = hh & 1;
+                if (!mbar_wait_bounded(&tma_bar[st], (hh >> 1) & 1)) {  // the issuer's wait then expires too
+                    if (lane == 0) atomicOr(&g_select_tc_errors, 4u);
+                    break;
+                }
+                qcal_rows(base + st * kStageBytes, wsm, 16 * (warp - 8), lane);
+                fence_async_smem();  // generic-proxy writes -> visible to the tensor core's operand reads
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&qcal_bar[st]);
+            }
+        }
     }
     // b' of the group's heads for chunks [0, 128), -inf beyond the summaries.
     for (int e = tid; e < 4 * kRows; e += blockDim.x) {
@@ -321,12 +416,39 @@ cudaError_t launch_select_tc(const Dims &D, const void *q_hat, const void *k_sum
     dim3 grid((D.T + kRows - 1) / kRows, D.Hkv, D.B);
     if (D.topk <= 16) {
         const size_t smem = 1024 + 2 * (size_t)kStageBytes;  // lists: 128 * 69 * 8 = 69 KiB fit in the stages
-        cudaFuncSetAttribute(select_tc_kernel<17, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        select_tc_kernel<17, 0><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap, nullptr, nullptr);
+        cudaFuncSetAttribute(select_tc_kernel<17, 0, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        select_tc_kernel<17, 0, 0><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap, nullptr, nullptr,
+                                                                     nullptr, nullptr);
     } else {
         const size_t smem = 1024 + (size_t)kRows * (4 * 33 + 1) * 8;  // 133 KiB of lists > the two stages
-        cudaFuncSetAttribute(select_tc_kernel<33, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        select_tc_kernel<33, 0><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap, nullptr, nullptr);
+        cudaFuncSetAttribute(select_tc_kernel<33, 0, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        select_tc_kernel<33, 0, 0><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap, nullptr, nullptr,
+                                                                     nullptr, nullptr);
+    }
+    return cudaGetLastError();
+}
+
+// The same selection from q with the Q-Cal projection fused in (rank 32, one W_down [32, 128] and
+// W_up [128, 32] pair for every head, bf16, 16-byte aligned).
+cudaError_t launch_select_tc_qcal(const Dims &D, const void *q, const void *w_down, const void *w_up,
+                                  const void *k_sum, const float *b_sum, int *idx, float *gap, cudaStream_t stream) {
+    CUtensorMap qmap, kmap;
+    if (!make_tmap_bf16_2d(&qmap, q, (uint64_t)D.B * D.Hq * D.T, 128, 128, 128) ||
+        !make_tmap_bf16_2d(&kmap, k_sum, (uint64_t)D.B * D.Hq * D.Nc, 128, 128, 128))
+        return cudaErrorInvalidValue;
+    dim3 grid((D.T + kRows - 1) / kRows, D.Hkv, D.B);
+    const auto *wd = (const __nv_bfloat16 *)w_down;
+    const auto *wu = (const __nv_bfloat16 *)w_up;
+    if (D.topk <= 16) {
+        const size_t smem = 1024 + 2 * (size_t)kStageBytes;
+        cudaFuncSetAttribute(select_tc_kernel<17, 0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        select_tc_kernel<17, 0, 1><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap, nullptr, nullptr,
+                                                                     wd, wu);
+    } else {
+        const size_t smem = 1024 + (size_t)kRows * (4 * 33 + 1) * 8;
+        cudaFuncSetAttribute(select_tc_kernel<33, 0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        select_tc_kernel<33, 0, 1><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap, nullptr, nullptr,
+                                                                     wd, wu);
     }
     return cudaGetLastError();
 }
@@ -341,9 +463,9 @@ cudaError_t launch_gather_shat_tc(const Dims &D, const void *q_hat, const void *
         return cudaErrorInvalidValue;
     dim3 grid((D.T + kRows - 1) / kRows, D.Hkv, D.B);
     const size_t smem = 1024 + 2 * (size_t)kStageBytes;
-    cudaFuncSetAttribute(select_tc_kernel<17, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    select_tc_kernel<17, 1><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, const_cast<int *>(idx), nullptr,
-                                                               ws_idx, ws_shat);
+    cudaFuncSetAttribute(select_tc_kernel<17, 1, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    select_tc_kernel<17, 1, 0><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, const_cast<int *>(idx), nullptr,
+                                                                  ws_idx, ws_shat, nullptr, nullptr);
     return cudaGetLastError();
 }
 

@@ -27,7 +27,7 @@ OP_SUMMARY, OP_SELECT, OP_ATTN_FWD, OP_DECODE, OP_ATTN_BWD = 0, 1, 2, 3, 4
 
 # Every symbol include/hils.h declares (checked by the tests against the header and the library).
 EXPORTED = ("hils_workspace_size", "hils_chunk_summary", "hils_chunk_summary_shared_query", "hils_select_topk",
-            "hils_bsa_select_topk", "hils_attn_fwd", "hils_decode", "hils_attn_bwd", "hils_check", "hils_status_string", "hils_last_error",
+            "hils_select_topk_qcal", "hils_bsa_select_topk", "hils_attn_fwd", "hils_decode", "hils_attn_bwd", "hils_check", "hils_status_string", "hils_last_error",
             "hils_version", "hils_decode_noalloc")
 
 
@@ -58,6 +58,8 @@ def _load() -> ctypes.CDLL:
     lib.hils_select_topk.restype = st
     lib.hils_bsa_select_topk.argtypes = [P, vp, vp, vp, vp, vp, vp]
     lib.hils_bsa_select_topk.restype = st
+    lib.hils_select_topk_qcal.argtypes = [P, vp, vp, vp, ctypes.c_int32, vp, vp, vp, vp, vp]
+    lib.hils_select_topk_qcal.restype = st
     lib.hils_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.hils_attn_fwd.restype = st
     lib.hils_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
@@ -193,6 +195,31 @@ def select_topk(q_hat, k_sum, b_sum, *, Hkv: int, L: int, S: int, topk: int, win
     ws, nws = _workspace(p, OP_SELECT, dev, None)
     _raise(lib.hils_select_topk(ctypes.byref(p), _ptr(q_hat), _ptr(k_sum), _ptr(b_sum), _ptr(idx), _ptr(gap),
                                 _ptr(ws), nws, _stream(dev)))
+    return (idx, gap) if gap is not None else idx
+
+
+def select_topk_qcal(q, w_down, w_up, k_sum, b_sum, *, Hkv: int, L: int, S: int, topk: int, window: int,
+                     q_pos0: int = 0, scale: float = 0.0, with_gap: bool = False, idx=None, gap=None):
+    """select_topk with Q-Cal fused (Sec. 4): q [B,Hq,T,d], w_down [r,d], w_up [d,r] (r = 32) ->
+    idx [B,Hkv,T,topk] int32 (and gap), selected on q^ = q + W_up (W_down q)."""
+    B, Hq, T, d = q.shape
+    dev, dt = q.device, q.dtype
+    r = w_down.shape[0]
+    _check("w_down", w_down, dt, (r, d), dev)
+    _check("w_up", w_up, dt, (d, r), dev)
+    Nc = L // S
+    _check("k_sum", k_sum, dt, (B, Hq, Nc, d), dev)
+    _check("b_sum", b_sum, torch.float32, (B, Hq, Nc), dev)
+    if idx is None:
+        idx = torch.empty((B, Hkv, T, topk), dtype=torch.int32, device=dev)
+    _check("idx", idx, torch.int32, (B, Hkv, T, topk), dev)
+    if with_gap and gap is None:
+        gap = torch.empty((B, Hkv, T), dtype=torch.float32, device=dev)
+    if gap is not None:
+        _check("gap", gap, torch.float32, (B, Hkv, T), dev)
+    p = make_params(B, T, L, Hq, Hkv, d, S, topk, window, q_pos0, scale, dt)
+    _raise(lib.hils_select_topk_qcal(ctypes.byref(p), _ptr(q), _ptr(w_down), _ptr(w_up), r, _ptr(k_sum), _ptr(b_sum),
+                                     _ptr(idx), _ptr(gap), _stream(dev)))
     return (idx, gap) if gap is not None else idx
 
 

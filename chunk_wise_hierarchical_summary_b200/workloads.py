@@ -81,15 +81,17 @@ def _randn(shape, g, device) -> torch.Tensor:
     return torch.randn(*shape, generator=g, device=device, dtype=torch.float32)
 
 
-def _qcal(q: torch.Tensor, d: int, g, device) -> torch.Tensor:
-    """q^ = q + W_up (W_down q), rank 32, weights N(0, 1/128) (input recipe, upstream of the path)."""
+def _qcal(q: torch.Tensor, d: int, g, device):
+    """q^ = q + W_up (W_down q), rank 32, weights N(0, 1/128) (input recipe, upstream of the path).
+    Returns (q^, W_down [32, d], W_up [d, 32])."""
     w_down = _randn((32, d), g, device) * math.sqrt(1.0 / 128.0)
     w_up = _randn((d, 32), g, device) * math.sqrt(1.0 / 128.0)
-    return q + (q @ w_down.t()) @ w_up.t()
+    return q + (q @ w_down.t()) @ w_up.t(), w_down, w_up
 
 
 def prefill_inputs(w: Workload, seed: int = 0, device="cpu", with_dout: bool = False) -> dict:
-    """q, q_hat [B,Hq,T,d]; k, v [B,Hkv,L,d]; q_land [B,Hq,Nc,d]; optional dout [B,Hq,T,d]."""
+    """q, q_hat [B,Hq,T,d]; k, v [B,Hkv,L,d]; q_land [B,Hq,Nc,d]; optional dout [B,Hq,T,d]; with the
+    "scaled" recipe also the Q-Cal weights that made q_hat, w_down [32,d] and w_up [d,32]."""
     g = _gen(seed, device)
     B, T, L, Hq, Hkv, d, Nc = w.B, w.T, w.L, w.Hq, w.Hkv, w.d, w.Nc
     if w.recipe == "tiny":
@@ -104,10 +106,12 @@ def prefill_inputs(w: Workload, seed: int = 0, device="cpu", with_dout: bool = F
         k = _randn((B, Hkv, L, d), g, device) * s
         v = _randn((B, Hkv, L, d), g, device) * s
         q_land = _randn((B, Hq, Nc, d), g, device)
-        q_hat = _qcal(q, d, g, device)
+        q_hat, w_down, w_up = _qcal(q, d, g, device)
     else:
         raise ValueError(f"prefill recipe {w.recipe!r}")
     out = {"q": q, "k": k, "v": v, "q_land": q_land, "q_hat": q_hat}
+    if w.recipe == "scaled":
+        out.update(w_down=w_down, w_up=w_up)
     if with_dout:
         out["dout"] = _randn((B, Hq, T, d), g, device)
     return {name: t.to(w.torch_dtype).contiguous() for name, t in out.items()}
@@ -125,7 +129,7 @@ def decode_inputs(w: Workload, seed: int = 0, device="cpu") -> dict:
     dt = w.torch_dtype
     q = _randn((B, Hq, w.T, d), g, device)
     q_land = _randn((B, Hq, w.Nc, d), g, device)
-    q_hat = _qcal(q, d, g, device)
+    q_hat, _, _ = _qcal(q, d, g, device)
     left = max(0, L - 1 - w.W + 1) // S * S
     n_cand = left // S
     n_needle = min(w.needles, n_cand)

@@ -121,6 +121,19 @@ HILS_API hils_status hils_select_topk(const hils_params *p, const void *q_hat, c
                              hils_stream_t stream);
 
 /*
+ * hils_select_topk with the Q-Cal projection (Sec. 4) fused into the score kernel: the retrieval query
+ * is q^ = q + W_up (W_down q) (rank 32, the token's own query as h, one pair shared by all heads), formed
+ * tile by tile in shared memory; no q^ tensor is read or written. q [B, Hq, T, d]; w_down [32, d] and
+ * w_up [d, 32] row-major, params.dtype, 16-byte aligned. Outputs, layouts and errors as
+ * hils_select_topk. Only the tensor-core shapes (bf16, d 128, G <= 4, topk <= 32, 1..128 candidates per
+ * row) and rank 32 are taken (HILS_ERR_UNSUPPORTED otherwise: form q^ and call hils_select_topk).
+ * No workspace.
+ */
+HILS_API hils_status hils_select_topk_qcal(const hils_params *p, const void *q, const void *w_down, const void *w_up,
+                                           int32_t rank, const void *k_sum, const float *b_sum, int32_t *idx,
+                                           float *gap, hils_stream_t stream);
+
+/*
  * Naive block-sparse attention selection (Sec. 2), the exact counterpart of hils_select_topk: for every
  * (b, query head h, row i) at position p with n = n_p candidates, the exact chunk mass
  *   mass[b,h,i,c] = LSE_{j in chunk c} tau q[b,h,i].k[b,h/G,j]   for c < n (entries c >= n untouched),

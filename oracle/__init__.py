@@ -8,6 +8,7 @@ statement in hils_oracle.c, which cites the paper section / equation each step f
   chunk_summary  Eq. 8 (Prop. 3.1)            select_topk  Sec. 3 RQ1 + Sec. 4 GQA selection
   chunk_summary_shared_query  Eq. 8 with one landmark query per head (Sec. 4)
   bsa_select_topk  naive BSA (Sec. 2): exact chunk masses, same group top-k
+  qcal, select_topk_qcal  Sec. 4 Q-Cal (q^ = q + W_up W_down q), then select_topk
   attn_fwd       Eq. 10, chunked form          eq10_tokenwise  Eq. 10, token by token
   attn_bwd       gradients of the above with the selection held fixed
   decode         select_topk + attn_fwd for one query at position L-1
@@ -159,6 +160,18 @@ def select_topk(g: Geometry, q_hat, k_sum, b_sum):
     gap = np.zeros((g.B, g.Hkv, g.T))
     _load().orc_select_topk(ctypes.byref(g._c()), _pd(qh), _pd(ks), _pd(bs), _pi(idx), _pd(gap))
     return idx, gap
+
+
+def qcal(q, w_down, w_up):
+    """Sec. 4 Q-Cal with the token's own query as h: q^ = q + W_up (W_down q), applied to every row
+    (last axis) of q; w_down [r, d], w_up [d, r]."""
+    q = np.asarray(q, dtype=np.float64)
+    return q + (q @ np.asarray(w_down, dtype=np.float64).T) @ np.asarray(w_up, dtype=np.float64).T
+
+
+def select_topk_qcal(g: Geometry, q, w_down, w_up, k_sum, b_sum):
+    """select_topk on the calibrated query q^ = qcal(q, w_down, w_up)."""
+    return select_topk(g, qcal(_f64(q, (g.B, g.Hq, g.T, g.d)), w_down, w_up), k_sum, b_sum)
 
 
 def bsa_select_topk(g: Geometry, q, k):

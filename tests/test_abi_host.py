@@ -124,6 +124,18 @@ def test_shared_query_summary_checked():
     assert H.lib.hils_chunk_summary_shared_query(ctypes.byref(p), None, None, 3, 3, None, None, None) == 0
 
 
+def test_fused_qcal_rules():
+    p = P()
+    st = H.lib.hils_select_topk_qcal(ctypes.byref(p), FAKE, FAKE, FAKE, 16, FAKE, FAKE, FAKE, None, None)
+    assert st == 2 and b"rank 16" in H.lib.hils_last_error()
+    p = P(dtype=1)
+    st = H.lib.hils_select_topk_qcal(ctypes.byref(p), FAKE, FAKE, FAKE, 32, FAKE, FAKE, FAKE, None, None)
+    assert st == 2 and b"hils_select_topk" in H.lib.hils_last_error()
+    p = P()
+    st = H.lib.hils_select_topk_qcal(ctypes.byref(p), FAKE, None, FAKE, 32, FAKE, FAKE, FAKE, None, None)
+    assert st == 1 and b"w_down is NULL" in H.lib.hils_last_error()
+
+
 def test_bsa_select_rules():
     p = P(topk=33)
     st = H.lib.hils_bsa_select_topk(ctypes.byref(p), FAKE, FAKE, FAKE, None, FAKE, None)

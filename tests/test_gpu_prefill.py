@@ -173,3 +173,50 @@ def test_chunk_summary_shared_query(dtype, Hq, Hkv, d, S, L):
     H.chunk_summary_shared_query(k.cuda(), qs.cuda(), S, c_begin=3, c_end=7, k_sum=ks2, b_sum=bs2)
     assert torch.equal(ks2[:, :, 3:7], ks[:, :, 3:7]) and torch.equal(bs2[:, :, 3:7], bs[:, :, 3:7])
     assert bool((ks2[:, :, :3] == 7).all()) and bool((bs2[:, :, 7:] == 7).all())
+
+
+@pytest.mark.parametrize("w", [
+    W.Workload("qcal_g4_k16", B=2, T=1000, L=1000, Hq=8, Hkv=2, d=128, S=64, topk=4, W=128, dtype="bf16",
+               recipe="scaled"),
+    W.Workload("qcal_g2_k32", B=1, T=2000, L=2000, Hq=4, Hkv=2, d=128, S=32, topk=20, W=256, dtype="bf16",
+               recipe="scaled"),
+    W.Workload("qcal_g1_offset", B=1, T=300, L=2300, Hq=2, Hkv=2, d=128, S=64, topk=6, W=64, dtype="bf16",
+               recipe="scaled", q_pos0=2000),
+], ids=lambda w: w.name)
+def test_select_fused_qcal(w):
+    """Selection with Q-Cal fused into the score kernel (q^ = q + W_up W_down q formed in shared memory)
+    against the oracle's Q-Cal + selection on the same bf16 q and weights; the unfused call on a q^ made
+    the same way agrees outside near ties."""
+    x = W.prefill_inputs(w, seed=9)
+    x["q"] = (x["q"].float() * 4).to(x["q"].dtype)  # wider score gaps: fewer rows inside the tie band
+    g = geometry(w)
+    xd = {n: t.cuda() for n, t in x.items()}
+    k_sum, b_sum = H.chunk_summary(xd["k"], xd["q_land"], w.S)
+    ridx, rgap = oracle.select_topk_qcal(g, np64(x["q"]), np64(x["w_down"]), np64(x["w_up"]), np64(k_sum),
+                                         np64(b_sum))
+    idx, gap = H.select_topk_qcal(xd["q"], xd["w_down"], xd["w_up"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S,
+                                  topk=w.topk, window=w.W, q_pos0=w.q_pos0, with_gap=True)
+    near = check_idx(idx, ridx, rgap)
+    assert near.mean() < 0.25
+    finite = np.isfinite(rgap)
+    assert_close(gap.cpu().numpy()[finite], rgap[finite], dict(atol=2e-3, rtol=2e-3), "gap")
+
+
+def test_select_fused_qcal_full_size_sampled():
+    """The prefill workload (B4 T8192 Hq16 Hkv4 d128 S64 k16 W512) with fused Q-Cal: ids of sampled 128-row
+    blocks against the oracle on the GPU's summaries."""
+    w = W.PREFILL_BF16
+    x = W.prefill_inputs(w, seed=0, device="cuda")
+    k_sum, b_sum = H.chunk_summary(x["k"], x["q_land"], w.S)
+    idx = H.select_topk_qcal(x["q"], x["w_down"], x["w_up"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S, topk=w.topk,
+                             window=w.W)
+    torch.cuda.synchronize()
+    wd, wu = np64(x["w_down"]), np64(x["w_up"])
+    for b, grp in ((1, 0), (2, 3)):
+        hs = slice(grp * w.G, (grp + 1) * w.G)
+        for r0 in (640, 8192 - 128):
+            gr = Geometry(B=1, T=128, L=w.L, Hq=w.G, Hkv=1, d=w.d, S=w.S, topk=w.topk, W=w.W, q_pos0=r0)
+            rows = slice(r0, r0 + 128)
+            ridx, rgap = oracle.select_topk_qcal(gr, np64(x["q"][b:b + 1, hs, rows]), wd, wu,
+                                                 np64(k_sum[b:b + 1, hs]), np64(b_sum[b:b + 1, hs]))
+            check_idx(idx[b:b + 1, grp:grp + 1, rows], ridx, rgap, f"idx b{b} g{grp} r{r0}")

@@ -267,6 +267,33 @@ def test_select_head_group_mapping():
         np.testing.assert_array_equal(idx[:, grp:grp + 1], i1)
 
 
+# ---------------------------------------------------------------- Q-Cal (Sec. 4)
+
+def test_qcal_closed_forms():
+    """q^ = q + W_up W_down q: with W_up = 0 (or W_down = 0) q^ = q; with W_down = the first r unit rows and
+    W_up = a times their transpose, q^ scales the first r coordinates by 1 + a and keeps the rest (a rank-r
+    projector), so the fused selection equals select_topk on that q^."""
+    d, r = 16, 4
+    rr = rng(41)
+    q = rr.standard_normal((1, 2, 30, d))
+    wd, wu = rr.standard_normal((r, d)), rr.standard_normal((d, r))
+    np.testing.assert_array_equal(oracle.qcal(q, wd, np.zeros((d, r))), q)
+    np.testing.assert_array_equal(oracle.qcal(q, np.zeros((r, d)), wu), q)
+    e = np.eye(d)[:r]
+    expect = q.copy()
+    expect[..., :r] *= 1.5
+    np.testing.assert_allclose(oracle.qcal(q, e, 0.5 * e.T), expect, rtol=0, atol=1e-15)
+    g = Geometry(B=1, T=30, L=30, Hq=2, Hkv=1, d=d, S=4, topk=2, W=6)
+    ks, bs = oracle.chunk_summary(g, rr.standard_normal((1, 1, 30, d)), rr.standard_normal((1, 2, g.Nc, d)))
+    i1, g1 = oracle.select_topk_qcal(g, q, e, 0.5 * e.T, ks, bs)
+    i2, g2 = oracle.select_topk(g, expect, ks, bs)
+    np.testing.assert_array_equal(i1, i2)
+    np.testing.assert_allclose(g1, g2, rtol=1e-12)
+    # the correction is linear in q and of rank <= r
+    corr = oracle.qcal(q, wd, wu) - q
+    assert np.linalg.matrix_rank(corr.reshape(-1, d)) <= r
+
+
 # ---------------------------------------------------------------- naive BSA (Sec. 2)
 
 def test_bsa_masses_brute_force_and_mha_topk():
