@@ -587,6 +587,9 @@ def profile_case(args):
         if st == "select":
             fn = lambda: H.select_topk(x["q_hat"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S, topk=w.topk, window=w.W,
                                        idx=idx)
+        elif st == "select_qcal":
+            fn = lambda: H.select_topk_qcal(x["q"], x["w_down"], x["w_up"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S,
+                                            topk=w.topk, window=w.W, idx=idx)
         elif st == "bsa":
             mass = torch.empty((w.B, w.Hq, w.T, w.Nc), dtype=torch.float32, device=dev)
             fn = lambda: H.bsa_select_topk(x["q"], x["k"], S=w.S, topk=w.topk, window=w.W, idx=idx, mass=mass)
@@ -612,7 +615,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="hils", choices=("hils", "reference"))
     ap.add_argument("--quick", action="store_true", help="headline only (no decode sweep / training blocks)")
-    ap.add_argument("--profile", choices=("summary", "select", "attn", "decode", "bwd", "bsa"),
+    ap.add_argument("--profile", choices=("summary", "select", "select_qcal", "attn", "decode", "bwd", "bsa"),
                     help="run --steps untimed launches of one stage for an ncu capture; no bench line")
     args = ap.parse_args()
     if args.profile:

@@ -38,12 +38,6 @@ constexpr int kSelWarps = 8;
 
 __device__ unsigned int g_bsa_errors = 0;
 
-struct Bars {
-    // With two K stages and two S buffers, s_full[b] (the QK product of tile n, n % 2 == b, completed)
-    // also frees K stage b; s_free[b] (all 128 rows have read S buffer b) lets the next QK overwrite it.
-    uint64_t q_full, k_full[kStages], s_full[2], s_free[2], done;
-};
-
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 bsa_mass_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, Dims D,
                    float *__restrict__ mass) {
@@ -229,16 +223,9 @@ bsa_mass_kernel(Dims D, const T *__restrict__ q, const T *__restrict__ k, float 
     }
 }
 
-__device__ __forceinline__ uint64_t warp_min_u64(uint64_t x) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const uint64_t y = __shfl_xor_sync(0xffffffffu, x, o);
-        x = y < x ? y : x;
-    }
-    return x;
-}
-
 // Group top-k from the masses: one warp per (b, g, i); lane t holds candidates t, t+32, ... (VPL per lane).
+// Warp-wide minima of the 64-bit (score desc, id asc) keys use two 32-bit redux steps (high word, then
+// the low word among the lanes holding that high word).
 template <int VPL>
 __global__ void __launch_bounds__(32 * kSelWarps)
 bsa_select_kernel(Dims D, const float *__restrict__ mass, int *__restrict__ idx, float *__restrict__ gap) {
@@ -248,7 +235,7 @@ bsa_select_kernel(Dims D, const float *__restrict__ mass, int *__restrict__ idx,
     const int i = (int)(w % D.T);
     const int g = (int)((w / D.T) % D.Hkv), b = (int)(w / ((long long)D.T * D.Hkv));
     const int n = window_left(D.q_pos0 + i, D.W, D.S) / D.S;
-    const int K = D.topk;
+    const int K = D.topk, G = D.G;
     int *out = idx + (size_t)w * K;
     if (n == 0) {
         if (lane < K) out[lane] = -1;
@@ -258,55 +245,74 @@ bsa_select_kernel(Dims D, const float *__restrict__ mass, int *__restrict__ idx,
     float gs[VPL];
 #pragma unroll
     for (int t = 0; t < VPL; ++t) gs[t] = -INFINITY;
-    for (int hh = 0; hh < D.G; ++hh) {
-        const float *mr = mass + (((size_t)b * D.Hq + g * D.G + hh) * D.T + i) * D.Nc;
-        float v[VPL];
-        float mx = -INFINITY;
+    // four heads at a time: their loads are in flight together and their reductions interleave
+    for (int h0 = 0; h0 < G; h0 += 4) {
+        float v[4][VPL], mx[4], z[4];
 #pragma unroll
-        for (int t = 0; t < VPL; ++t) {
-            const int c = lane + 32 * t;
-            v[t] = c < n ? __ldg(mr + c) : -INFINITY;
-            mx = fmaxf(mx, v[t]);
-        }
-        mx = warp_max(mx);
-        float z = 0.f;
+        for (int u = 0; u < 4; ++u) {
+            const bool live = h0 + u < G;
+            const float *mr = mass + (((size_t)b * D.Hq + g * G + h0 + (live ? u : 0)) * D.T + i) * D.Nc;
+            mx[u] = -INFINITY;
 #pragma unroll
-        for (int t = 0; t < VPL; ++t) z += (lane + 32 * t < n) ? __expf(v[t] - mx) : 0.f;
-        const float lse = mx + __logf(warp_sum(z));
-#pragma unroll
-        for (int t = 0; t < VPL; ++t)
-            if (lane + 32 * t < n) gs[t] = fmaxf(gs[t], v[t] - lse);
-    }
-    // rounds of warp-wide (score desc, id asc) minimum; the winner's lane retires the entry
-    uint32_t taken = 0;
-    auto lane_best = [&]() {
-        uint64_t best = ~0ull;
-#pragma unroll
-        for (int t = 0; t < VPL; ++t) {
-            const int c = lane + 32 * t;
-            if (c < n && !((taken >> t) & 1u)) {
-                const uint64_t key = desc_value_key(gs[t], (uint32_t)c);
-                best = key < best ? key : best;
+            for (int t = 0; t < VPL; ++t) {
+                const int c = lane + 32 * t;
+                v[u][t] = (live && c < n) ? __ldg(mr + c) : -INFINITY;
             }
         }
-        return best;
-    };
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+#pragma unroll
+            for (int t = 0; t < VPL; ++t) mx[u] = fmaxf(mx[u], v[u][t]);
+            mx[u] = float_from_order_key(__reduce_max_sync(0xffffffffu, float_order_key(mx[u])));
+            z[u] = 0.f;
+#pragma unroll
+            for (int t = 0; t < VPL; ++t) z[u] += (v[u][t] > -INFINITY) ? __expf(v[u][t] - mx[u]) : 0.f;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) z[u] += __shfl_xor_sync(0xffffffffu, z[u], o);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (h0 + u >= G) break;
+            const float lse = mx[u] + __logf(z[u]);
+#pragma unroll
+            for (int t = 0; t < VPL; ++t)
+                if (lane + 32 * t < n) gs[t] = fmaxf(gs[t], v[u][t] - lse);
+        }
+    }
+    uint64_t key[VPL];
+#pragma unroll
+    for (int t = 0; t < VPL; ++t) {
+        const int c = lane + 32 * t;
+        key[t] = c < n ? desc_value_key(gs[t], (uint32_t)c) : ~0ull;
+    }
     const int kk = min(K, n);
     const int rounds = kk + (n > K ? 1 : 0);
     int my_id = -1;
     float s_k = 0.f, s_k1 = 0.f;
     for (int rd = 0; rd < rounds; ++rd) {
-        const uint64_t best = warp_min_u64(lane_best());
-        const int c = (int)desc_key_index(best);
+        uint64_t best = key[0];
+#pragma unroll
+        for (int t = 1; t < VPL; ++t) best = key[t] < best ? key[t] : best;
+        const uint32_t hi = (uint32_t)(best >> 32);
+        const uint32_t bh = __reduce_min_sync(0xffffffffu, hi);
+        const uint32_t bl = __reduce_min_sync(0xffffffffu, hi == bh ? (uint32_t)best : 0xffffffffu);
+        const int c = (int)bl;
+        const float sv = float_from_order_key(~bh);
         if (rd < kk && lane == rd) my_id = c;
-        if (rd == kk - 1) s_k = desc_key_value(best);
-        if (rd == kk) s_k1 = desc_key_value(best);
-        if ((c & 31) == lane) taken |= 1u << (c >> 5);
+        if (rd == kk - 1) s_k = sv;
+        if (rd == kk) s_k1 = sv;
+        if ((c & 31) == lane) {
+#pragma unroll
+            for (int t = 0; t < VPL; ++t)
+                if (t == (c >> 5)) key[t] = ~0ull;
+        }
     }
     // ids ascending: the lane holding the r-th winner finds its rank among the kk winners
     int rank = 0;
-    for (int s = 0; s < kk; ++s) {
-        const int o = __shfl_sync(0xffffffffu, my_id, s);
+    for (int s2 = 0; s2 < kk; ++s2) {
+        const int o = __shfl_sync(0xffffffffu, my_id, s2);
         rank += (lane < kk && o < my_id) ? 1 : 0;
     }
     if (lane < kk) out[rank] = my_id;
