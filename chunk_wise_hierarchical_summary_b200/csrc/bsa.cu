@@ -38,6 +38,12 @@ constexpr int kSelWarps = 8;
 
 __device__ unsigned int g_bsa_errors = 0;
 
+struct Bars {
+    // With two K stages and two S buffers, s_full[b] (the QK product of tile n, n % 2 == b, completed)
+    // also frees K stage b; s_free[b] (all 128 rows have read S buffer b) lets the next QK overwrite it.
+    uint64_t q_full, k_full[kStages], s_full[2], s_free[2], done;
+};
+
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 bsa_mass_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, Dims D,
                    float *__restrict__ mass) {
