@@ -585,8 +585,14 @@ decode_select_warp_kernel(Dims D, DecodePlan P, const float *__restrict__ scores
     constexpr int kSelWPer = 64 / GM;                     // candidates per thread per round
     constexpr int kSelWRound = kSelWThreads * kSelWPer;
     const int rounds = (n + kSelWRound - 1) / kSelWRound;
-    // candidate of (round r, slot i) for this thread: coalesced across the warp
-    auto cand = [&](int r, int i) { return r * kSelWRound + warp * (32 * kSelWPer) + i * 32 + lane; };
+    // candidate of (round r, slot i) for this thread, coalesced across the warp. A list shorter than one
+    // round is spread over all threads, so that every thread holds its own best key (held by a few warps
+    // it would leave the 32nd-best bound loose and overflow the survivor buffer); longer lists give each
+    // warp a contiguous block per round.
+    const bool spread = n < kSelWRound;
+    auto cand = [&](int r, int i) {
+        return spread ? i * kSelWThreads + tid : r * kSelWRound + warp * (32 * kSelWPer) + i * 32 + lane;
+    };
     float raw[GM][kSelWPer];
     auto load_round = [&](int r) {
 #pragma unroll
