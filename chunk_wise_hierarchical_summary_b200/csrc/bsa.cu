@@ -14,8 +14,6 @@
 //     bsa_mass_kernel (any dtype and shape): one warp per (b, h, i), lanes split d.
 //  2. bsa_select_kernel: one warp per (b, g, i) reads the G heads' masses of its row and runs the
 //     group top-k with (score desc, id asc) 64-bit keys.
-#include <climits>
-
 #include "internal.h"
 #include "tcgen05.cuh"
 
