@@ -585,11 +585,11 @@ decode_select_warp_kernel(Dims D, DecodePlan P, const float *__restrict__ scores
     constexpr int kSelWPer = 64 / GM;                     // candidates per thread per round
     constexpr int kSelWRound = kSelWThreads * kSelWPer;
     const int rounds = (n + kSelWRound - 1) / kSelWRound;
-    // candidate of (round r, slot i) for this thread, coalesced across the warp. A list shorter than one
-    // round is spread over all threads, so that every thread holds its own best key (held by a few warps
+    // candidate of (round r, slot i) for this thread, coalesced across the warp. A list shorter than half
+    // a round is spread over all threads, so that every thread holds its own best key (held by a few warps
     // it would leave the 32nd-best bound loose and overflow the survivor buffer); longer lists give each
-    // warp a contiguous block per round.
-    const bool spread = n < kSelWRound;
+    // warp a contiguous block per round (eight or more warps then hold candidates).
+    const bool spread = n < kSelWRound / 2;
     auto cand = [&](int r, int i) {
         return spread ? i * kSelWThreads + tid : r * kSelWRound + warp * (32 * kSelWPer) + i * 32 + lane;
     };
@@ -951,10 +951,14 @@ cudaError_t launch_t(const Dims &D, const void *q, const void *q_hat, const void
                                                            part);
     }
     unsigned int *selcount = (unsigned int *)(w + P.off_selcount);
-    if (D.topk <= 32 && D.G <= 4)
+    // One CTA per (b, KV group, query) selects the top-k of a whole candidate list. With few groups and a
+    // long list (a few sequences over a multi-million-token cache) that leaves most SMs idle: the list is
+    // then split over ceil(n / 1024) CTAs per group whose top-(k+1) lists the last CTA merges.
+    const bool wide = D.T == 1 && D.B * D.Hkv < 32 && P.n >= 16384 && next_pow2(P.nparts * D.topk) <= kSelMerge;
+    if (!wide && D.topk <= 32 && D.G <= 4)
         decode_select_warp_kernel<4><<<dim3(D.Hkv, D.B * D.T), kSelWThreads, 0, stream>>>(D, P, scores, part, sel,
                                                                                           idx_out);
-    else if (D.topk <= 32 && D.G <= 8)
+    else if (!wide && D.topk <= 32 && D.G <= 8)
         decode_select_warp_kernel<8><<<dim3(D.Hkv, D.B * D.T), kSelWThreads, 0, stream>>>(D, P, scores, part, sel,
                                                                                           idx_out);
     else

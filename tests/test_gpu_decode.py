@@ -56,6 +56,9 @@ def check_groups(w, x, k_sum, b_sum, out, lse, idx, groups):
                recipe="needle", q_pos0=4999, needles=5),
     W.Workload("dec_g1", B=1, T=1, L=3000, Hq=3, Hkv=3, d=128, S=64, topk=8, W=200, dtype="bf16",
                recipe="needle", q_pos0=2999, needles=3),
+    # one KV group over a 1M-token cache (16385 candidates): the list is split over several selection CTAs
+    W.Workload("dec_long_one_group", B=1, T=1, L=1049176, Hq=4, Hkv=1, d=128, S=64, topk=8, W=512, dtype="bf16",
+               recipe="needle", q_pos0=1049175, needles=4),
 ], ids=lambda w: w.name)
 def test_decode_shapes(w):
     x = W.decode_inputs(w, seed=1, device="cpu")
