@@ -149,6 +149,12 @@ def test_decode_select_periodic_scores():
                recipe="needle", q_pos0=4992, needles=5),
     W.Workload("dec_m2_g1", B=3, T=2, L=3000, Hq=4, Hkv=4, d=128, S=64, topk=8, W=200, dtype="bf16",
                recipe="needle", q_pos0=2998, needles=3),
+    # topk >= every query's candidates: the last two queries select chunk 10, which lies in the first two
+    # queries' windows (a union tile that is a window tile for some rows and a selected chunk for others)
+    W.Workload("dec_m4_window_and_selected", B=1, T=4, L=961, Hq=8, Hkv=2, d=128, S=64, topk=16, W=256,
+               dtype="bf16", recipe="needle", q_pos0=957, needles=2),
+    W.Workload("dec_m8_g4", B=2, T=8, L=7000, Hq=8, Hkv=2, d=128, S=64, topk=16, W=200, dtype="bf16",
+               recipe="needle", q_pos0=6992, needles=5),
 ], ids=lambda w: w.name)
 def test_multi_token_decode(w):
     """M query tokens at the end of the cache in one decode call: per query its own candidates, top-k
