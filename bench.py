@@ -193,6 +193,17 @@ def timed_steps(steps, fn_stages, warmup, flush, dist: Dist, sampler=None):
     return stage_ms, sum(stage_ms), clocks
 
 
+# ----------------------------------------------------------------------------- the line both arms print
+
+METRIC = ("HiLS prefill tokens/s (B4 T8192 Hq16 Hkv4 d128 S64 k16 W512); decode us/token at 512K ctx in 'decode'; "
+          "% of TC/HBM roofline")
+
+
+def base_config(w: W.Workload, world: int) -> dict:
+    return {"workload": w.name, "global_batch": w.B * world, "seq_len": w.T,
+            "parallelism": f"dp{world} (independent sequences per GPU)"}
+
+
 # ----------------------------------------------------------------------------- algorithmic work
 
 def window_left(p, Wn, S):
@@ -547,11 +558,11 @@ def run_reference(args, dist):
         tokens += t
     value = tokens / total
     sample = (f"1 (batch, KV group) slice x {blocks} blocks of {rows} query rows per step; tokens = rows*G/Hq")
-    line = {"metric": "HiLS prefill tokens/s (B4 T8192 Hq16 Hkv4 d128 S64 k16 W512)", "value": value,
+    line = {"metric": METRIC, "value": value,
             "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.T, "parallelism": "cpu oracle"},
+            "config": base_config(w, 1),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -658,13 +669,11 @@ def main():
             cpu = cpu_baseline(pre["x"], w)
         launches = pre["launches_per_step"] * args.steps
         line = {
-            "metric": "HiLS prefill tokens/s (B4 T8192 Hq16 Hkv4 d128 S64 k16 W512); decode us/token at 512K ctx in "
-                      "'decode'; % of TC/HBM roofline",
+            "metric": METRIC,
             "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": w.name, "global_batch": w.B * dist.world, "seq_len": w.T,
-                       "parallelism": f"dp{dist.world} (independent sequences per GPU)",
+            "config": {**base_config(w, dist.world),
                        "l2": "flushed (256 MiB write) between timed steps, outside the events",
                        "peaks": peak_src},
             "stage_ms": {"chunk_summary": pre["stage_ms"][0], "select_topk": pre["stage_ms"][1],
