@@ -199,6 +199,12 @@ METRIC = ("HiLS prefill tokens/s (B4 T8192 Hq16 Hkv4 d128 S64 k16 W512); decode 
           "% of TC/HBM roofline")
 
 
+# DRAM bytes (read + write) of one attn_tc_kernel launch at the prefill workload, from one ncu capture
+# (`--metrics dram__bytes_read.sum,dram__bytes_write.sum` of `bench.py --profile attn`): 241.7 MB read,
+# 102.2 MB written. Valid for the kernel as captured; set to None when the kernel changes.
+ATTN_TC_TRAFFIC_BYTES = 241742336 + 102183680
+
+
 def base_config(w: W.Workload, world: int) -> dict:
     return {"workload": w.name, "global_batch": w.B * world, "seq_len": w.T,
             "parallelism": f"dp{world} (independent sequences per GPU)"}
@@ -291,9 +297,10 @@ def bench_prefill(args, dist, dev, H, peaks):
         "ms_per_step": total_ms / args.steps, "clocks": clocks, "work": work,
         "roofline": {"bound": "tensor", "kernel": "hils_attn_fwd", "achieved": achieved,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                     "traffic": None,
+                     "traffic": ATTN_TC_TRAFFIC_BYTES,
                      "note": "algorithmic flops = 4*d per (row, head, attended token); attended = window + "
-                             "selected chunk tokens, %.1f per query on average" % work["avg_attended"]},
+                             "selected chunk tokens, %.1f per query on average; traffic = DRAM bytes per "
+                             "attn_tc_kernel launch (ncu)" % work["avg_attended"]},
         "launches_per_step": 3,
     }
     del flush

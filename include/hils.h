@@ -6,7 +6,10 @@
  * (Eq. 7) and GQA-shared top-k chunk selection (Sec. 3 RQ1, Sec. 4 "GQA"), (c) softmax attention of
  * each query within each selected chunk and within its chunk-aligned causal sliding window
  * (Sec. 2), (d) fusion of the per-chunk outputs by softmax(s^) over the selected chunks plus the
- * window (Eq. 10), in prefill, single-token decode and backward forms.
+ * window (Eq. 10), in prefill, decode (one or up to 8 query tokens) and backward forms. Beside them:
+ * stage (a) with one shared landmark query per head (Sec. 4), stage (b) with the Q-Cal projection
+ * fused in (Sec. 4), and the naive block-sparse selection on exact chunk masses (Sec. 2) as the
+ * reference for selection quality.
  *
  * Conventions shared by every call
  * --------------------------------
