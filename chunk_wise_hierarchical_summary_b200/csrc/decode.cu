@@ -952,9 +952,10 @@ cudaError_t launch_t(const Dims &D, const void *q, const void *q_hat, const void
     }
     unsigned int *selcount = (unsigned int *)(w + P.off_selcount);
     // One CTA per (b, KV group, query) selects the top-k of a whole candidate list. With few groups and a
-    // long list (a few sequences over a multi-million-token cache) that leaves most SMs idle: the list is
-    // then split over ceil(n / 1024) CTAs per group whose top-(k+1) lists the last CTA merges.
-    const bool wide = D.T == 1 && D.B * D.Hkv < 32 && P.n >= 16384 && next_pow2(P.nparts * D.topk) <= kSelMerge;
+    // long list (a few sequences over a cache of a million tokens or more) that leaves most SMs idle: the
+    // list is then split over ceil(n / 1024) CTAs per group whose top-(k+1) lists the last CTA merges.
+    // (Measured at B1: 8184 candidates faster on one CTA, 16376 and more faster split.)
+    const bool wide = D.T == 1 && D.B * D.Hkv < 32 && P.n >= 12288 && next_pow2(P.nparts * D.topk) <= kSelMerge;
     if (!wide && D.topk <= 32 && D.G <= 4)
         decode_select_warp_kernel<4><<<dim3(D.Hkv, D.B * D.T), kSelWThreads, 0, stream>>>(D, P, scores, part, sel,
                                                                                           idx_out);
