@@ -84,6 +84,30 @@ __device__ __forceinline__ void block_bitonic_sort(uint64_t *keys, int n) {
     __syncthreads();
 }
 
+// Programmatic dependent launch: a kernel launched with launch_pdl may start while the grid before it
+// on the stream is still running; grid_dep_wait() blocks until that grid has completed and its memory
+// is visible (a no-op for an ordinary launch). Every CTA of such a kernel calls it before reading what
+// the previous grid wrote and before it exits, so completion stays transitive along the chain.
+// grid_dep_launch() lets the next PDL-launched grid start early.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Number of SMs of the current device (cached per device ordinal).
 inline int num_sms() {
     static int cache[256] = {0};

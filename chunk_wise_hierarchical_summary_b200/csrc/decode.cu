@@ -120,6 +120,7 @@ decode_score_kernel(Dims D, DecodePlan P, const T *__restrict__ q_hat, const T *
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t slot_bytes = (size_t)P.per * d * sizeof(T);
     const int units = D.B * D.Hq * P.nslices;
+    grid_dep_launch();  // the selection's CTAs may take SMs as this grid's CTAs finish
     if (tid == 0) {
         for (int i = 0; i < NS; ++i) {
             mbar_init(&full[i], 1);
@@ -318,6 +319,7 @@ decode_select_kernel(Dims D, DecodePlan P, const float *__restrict__ scores, con
     const int G = D.G, K = D.topk, n = P.n;
     const size_t bg = (size_t)b * D.Hkv + g;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    grid_dep_wait();  // the score grid's scores and partials
     int *out = sel + bg * K;
     int *out2 = idx_out ? idx_out + bg * K : nullptr;
     if (n == 0) {
@@ -570,6 +572,7 @@ decode_select_warp_kernel(Dims D, DecodePlan P, const float *__restrict__ scores
     const int G = D.G, K = D.topk;
     const int n = window_left(D.q_pos0 + m, D.W, D.S) / D.S;
     const size_t bgm = ((size_t)b * D.Hkv + g) * M + m;
+    grid_dep_wait();  // the score grid's scores and partials
     const size_t hs = (size_t)M * P.n;  // stride between the group's heads in the score rows
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = kSelWThreads / 32;
     int *out = sel + bgm * K;
@@ -956,15 +959,20 @@ cudaError_t launch_t(const Dims &D, const void *q, const void *q_hat, const void
     // list is then split over ceil(n / 1024) CTAs per group whose top-(k+1) lists the last CTA merges.
     // (Measured at B1: 8184 candidates faster on one CTA, 16376 and more faster split.)
     const bool wide = D.T == 1 && D.B * D.Hkv < 32 && P.n >= 12288 && next_pow2(P.nparts * D.topk) <= kSelMerge;
+    cudaError_t es;
     if (!wide && D.topk <= 32 && D.G <= 4)
-        decode_select_warp_kernel<4><<<dim3(D.Hkv, D.B * D.T), kSelWThreads, 0, stream>>>(D, P, scores, part, sel,
-                                                                                          idx_out);
+        es = launch_pdl(decode_select_warp_kernel<4>, dim3(D.Hkv, D.B * D.T), dim3(kSelWThreads), 0, stream, D, P,
+                        (const float *)scores, (const float *)part, sel, idx_out);
     else if (!wide && D.topk <= 32 && D.G <= 8)
-        decode_select_warp_kernel<8><<<dim3(D.Hkv, D.B * D.T), kSelWThreads, 0, stream>>>(D, P, scores, part, sel,
-                                                                                          idx_out);
-    else
+        es = launch_pdl(decode_select_warp_kernel<8>, dim3(D.Hkv, D.B * D.T), dim3(kSelWThreads), 0, stream, D, P,
+                        (const float *)scores, (const float *)part, sel, idx_out);
+    else {
+        // an ordinary launch: started early behind the score grid this split form measured slower
         decode_select_kernel<<<dim3(P.nparts, D.Hkv, D.B), kSelThreads, 0, stream>>>(D, P, scores, part, lists,
                                                                                      selcount, sel, idx_out);
+        es = cudaGetLastError();
+    }
+    if (es != cudaSuccess) return es;
     if (decode_attn_mma_supported(D, sizeof(T) == 2 ? HILS_BF16 : HILS_FP32, q, k_cache, v_cache, P.ntiles))
         return launch_decode_attn_mma(D, P.n, P.ntiles, q, k_cache, v_cache, scores, sel, partial, counters, out, lse,
                                       stream);

@@ -69,6 +69,7 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     const size_t bgm = bg * M + m;            // this query's ids and counter
     const int pos = D.q_pos0 + m;
     const int l = window_left(pos, D.W, S);
+    grid_dep_wait();  // the selection grid's ids (and, through it, the scores)
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -352,10 +353,9 @@ cudaError_t launch_decode_attn_mma(const Dims &D, int n, int ntiles, const void 
     const size_t smem = 1024 + kStages * 2 * kTileBytes;
     cudaFuncSetAttribute(decode_attn_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     const int nsplit = decode_attn_mma_splits(D, ntiles);
-    decode_attn_mma_kernel<<<dim3(nsplit, D.Hkv, D.B * D.T), kThreads, smem, stream>>>(
-        kmap, vmap, D, n, ntiles, (const __nv_bfloat16 *)q, scores, sel, partial, counters, (__nv_bfloat16 *)out,
-        lse);
-    return cudaGetLastError();
+    return launch_pdl(decode_attn_mma_kernel, dim3(nsplit, D.Hkv, D.B * D.T), dim3(kThreads), smem, stream, kmap, vmap,
+                      D, n, ntiles, (const __nv_bfloat16 *)q, scores, sel, partial, counters, (__nv_bfloat16 *)out,
+                      lse);
 }
 
 }  // namespace hils

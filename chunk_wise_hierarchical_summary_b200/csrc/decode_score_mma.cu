@@ -45,6 +45,7 @@ decode_score_mma_kernel(const __grid_constant__ CUtensorMap kmap, Dims D, int n,
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int M = D.T;
     const long long units = (long long)D.B * D.Hq * nslices;
+    grid_dep_launch();  // the selection's CTAs may take SMs as this grid's CTAs finish
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
