@@ -166,22 +166,38 @@ def test_multi_token_decode(w):
                              window=w.W, return_idx=True)
     assert tuple(out.shape) == (w.B, w.Hq, w.T, w.d) and tuple(lse.shape) == (w.B, w.Hq, w.T)
     assert tuple(idx.shape) == (w.B, w.Hkv, w.T, w.topk)
+    check_multi_groups(w, x, out, lse, idx, [(b, g) for b in range(w.B) for g in range(w.Hkv)])
+
+
+def test_multi_token_decode_full_size_sampled():
+    """Multi-token decode at the decode workload's size (B8 L524288 Hq32 Hkv8 d128 S64 k32 W512, M = 4 query
+    tokens per sequence) on three (b, group) pairs against the oracle."""
+    w = W.DECODE_BF16.with_(name="decode_m4", T=4, q_pos0=W.DECODE_BF16.L - 4)
+    x = W.decode_inputs(w, seed=11, device="cuda")
+    k_sum, b_sum = H.chunk_summary(x["k_cache"], x["q_land"], w.S)
+    out, lse, idx = H.decode(x["q"], x["q_hat"], x["k_cache"], x["v_cache"], k_sum, b_sum, S=w.S, topk=w.topk,
+                             window=w.W, return_idx=True)
+    torch.cuda.synchronize()
+    check_multi_groups(w, x, out, lse, idx, [(0, 0), (5, 3), (7, 7)])
+
+
+def check_multi_groups(w, x, out, lse, idx, groups):
+    """Oracle evaluation of the M rows of the listed (b, group) pairs from the raw cache."""
     tol = TOL[w.dtype]
-    for b in range(w.B):
-        for grp in range(w.Hkv):
-            hs = slice(grp * w.G, (grp + 1) * w.G)
-            g1 = Geometry(B=1, T=w.T, L=w.L, Hq=w.G, Hkv=1, d=w.d, S=w.S, topk=w.topk, W=w.W, q_pos0=w.q_pos0)
-            kk = np64(x["k_cache"][b:b + 1, grp:grp + 1])
-            vv = np64(x["v_cache"][b:b + 1, grp:grp + 1])
-            rk, rb = oracle.chunk_summary(g1, kk, np64(x["q_land"][b:b + 1, hs]))
-            qh = np64(x["q_hat"][b:b + 1, hs])
-            ridx, rgap = oracle.select_topk(g1, qh, rk, rb)
-            near = check_idx(idx[b:b + 1, grp:grp + 1], ridx, rgap, f"multi idx b{b} g{grp}")
-            if near.any():
-                continue
-            ro, rl = oracle.attn_fwd(g1, np64(x["q"][b:b + 1, hs]), kk, vv, qh, rk, rb, ridx)
-            assert_close(out[b:b + 1, hs], ro, tol, f"multi out b{b} g{grp}")
-            assert_close(lse[b:b + 1, hs], np.asarray(rl).reshape(1, w.G, w.T), tol, f"multi lse b{b} g{grp}")
+    for b, grp in groups:
+        hs = slice(grp * w.G, (grp + 1) * w.G)
+        g1 = Geometry(B=1, T=w.T, L=w.L, Hq=w.G, Hkv=1, d=w.d, S=w.S, topk=w.topk, W=w.W, q_pos0=w.q_pos0)
+        kk = np64(x["k_cache"][b:b + 1, grp:grp + 1])
+        vv = np64(x["v_cache"][b:b + 1, grp:grp + 1])
+        rk, rb = oracle.chunk_summary(g1, kk, np64(x["q_land"][b:b + 1, hs]))
+        qh = np64(x["q_hat"][b:b + 1, hs])
+        ridx, rgap = oracle.select_topk(g1, qh, rk, rb)
+        near = check_idx(idx[b:b + 1, grp:grp + 1], ridx, rgap, f"multi idx b{b} g{grp}")
+        if near.any():
+            continue
+        ro, rl = oracle.attn_fwd(g1, np64(x["q"][b:b + 1, hs]), kk, vv, qh, rk, rb, ridx)
+        assert_close(out[b:b + 1, hs], ro, tol, f"multi out b{b} g{grp}")
+        assert_close(lse[b:b + 1, hs], np.asarray(rl).reshape(1, w.G, w.T), tol, f"multi lse b{b} g{grp}")
 
 
 def test_multi_token_decode_rows_match_single_token_at_last_position():
