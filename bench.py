@@ -462,6 +462,43 @@ def bench_select_qcal(args, dist, dev, H):
             "note": "fused: hils_select_topk_qcal from q, W_down, W_up; unfused: hils_select_topk from q^"}
 
 
+def bench_prefill_local(args, dist, dev, H, peaks):
+    """The prefill attention on position-correlated queries (recipe "local": adjacent queries select
+    overlapping chunks, the regime the query packing of Sec. 4 assumes), next to the union ratio of the
+    selections: chunks a 32-query tile visits (window and selected) per chunk one query attends."""
+    w = W.PREFILL_LOCAL_BF16
+    x = W.prefill_inputs(w, seed=rank_seed(1000, dist.rank), device=dev)
+    out, lse, idx, k_sum, b_sum = H.prefill(x["q"], x["k"], x["v"], x["q_hat"], x["q_land"], S=w.S, topk=w.topk,
+                                            window=w.W)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(mark):
+        H.attn_fwd(x["q"], x["k"], x["v"], x["q_hat"], k_sum, b_sum, idx, S=w.S, window=w.W, out=out, lse=lse)
+        mark()
+
+    steps = max(1, min(args.steps, 10))
+    _, total_ms, _ = timed_steps(steps, step, 3, flush, dist)
+    ms = dist.max(total_ms / steps)
+    work = prefill_work(w)
+    tf = work["attn_flops"] / (ms / 1e3) / 1e12
+    return {"workload": w.name, "attn_ms": ms, "achieved_tflops": tf, "frac": tf / peaks["bf16_tflops"],
+            **packing_stats(w, idx),
+            "note": "hils_attn_fwd alone on its own selection; algorithmic flops as in the headline"}
+
+
+def packing_stats(w: W.Workload, idx) -> dict:
+    """Selected chunks per query against distinct selected chunks per tile of 128 / G queries (the rows
+    one attention CTA packs): how much of a tile's selected-chunk work each row actually uses."""
+    QT = 128 // w.G
+    nt = w.T // QT
+    sel = idx[:, :, :nt * QT].reshape(w.B, w.Hkv, nt, QT * w.topk).long()
+    hit = torch.zeros((w.B, w.Hkv, nt, w.Nc + 1), dtype=torch.bool, device=idx.device)
+    hit.scatter_(3, torch.where(sel < 0, torch.full_like(sel, w.Nc), sel), True)
+    return {"selected_chunks_per_query": (idx >= 0).sum(-1).double().mean().item(),
+            "selected_chunks_per_tile": hit[..., :w.Nc].sum(-1).double().mean().item(),
+            "queries_per_tile": QT}
+
+
 def bench_train(args, dist, dev, H, peaks):
     w = W.TRAIN_BF16
     x = W.prefill_inputs(w, seed=rank_seed(3000, dist.rank), device=dev, with_dout=True)
@@ -671,6 +708,7 @@ def main():
             extra["train"] = bench_train(args, dist, dev, H, peaks)
             extra["bsa_select"] = bench_bsa(args, dist, dev, H, peaks)
             extra["select_qcal"] = bench_select_qcal(args, dist, dev, H)
+            extra["prefill_local"] = bench_prefill_local(args, dist, dev, H, peaks)
         cpu = None
         if dist.world == 1:
             cpu = cpu_baseline(pre["x"], w)
@@ -686,6 +724,7 @@ def main():
             "stage_ms": {"chunk_summary": pre["stage_ms"][0], "select_topk": pre["stage_ms"][1],
                          "attn_fwd": pre["stage_ms"][2]},
             "roofline": pre["roofline"],
+            "packing": packing_stats(w, pre["idx"]),
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches,

@@ -9,6 +9,9 @@ Recipes (paper: "Hierarchical Sparse Attention Done Right: Toward Infinite Conte
   scaled    q, k, v ~ N(0,1) * d**-0.25 (so q.k/sqrt(d) has std 1/sqrt(d)); q' ~ N(0,1);
             q^ = q + W_up (W_down q) with W_down [32,d], W_up [d,32] i.i.d. N(0, 1/128), one pair
             shared by every head (the Sec. 4 low-rank query calibration with h_i := q_i).
+  local     as scaled, but each head's q is a first-order autoregressive sequence along the positions,
+            q_i = rho q_(i-1) + sqrt(1 - rho^2) e_i (e_i i.i.d. N(0,1), rho = 0.995), so adjacent queries
+            are correlated and select overlapping chunks, the regime Sec. 4's query packing assumes.
   needle    decode cache: q, q' ~ N(0,1), q^ from q as above, K/V ~ N(0,1); 16 distinct candidate
             chunks per sequence hold "needle" keys 0.8*sqrt(d)*q^_h0/|q^_h0| + N(0, 0.2^2), h0 the
             first query head of each KV group.
@@ -34,7 +37,7 @@ class Workload:
     topk: int
     W: int
     dtype: str  # "fp32" or "bf16"
-    recipe: str  # "tiny", "scaled" or "needle"
+    recipe: str  # "tiny", "scaled", "local" or "needle"
     q_pos0: int = 0
     needles: int = 0
     extra: dict = field(default_factory=dict, compare=False)
@@ -63,6 +66,9 @@ PREFILL_BF16 = Workload("prefill_bf16_B4_T8192_Hq16_Hkv4_d128_S64_k16_W512", B=4
 DECODE_BF16 = Workload("decode_bf16_B8_L524288_Hq32_Hkv8_d128_S64_k32_W512", B=8, T=1, L=524288, Hq=32, Hkv=8,
                        d=128, S=64, topk=32, W=512, dtype="bf16", recipe="needle", q_pos0=524287, needles=16)
 DECODE_SWEEP_L = (32768, 131072, 524288, 1048576, 2097152, 4194304)
+# The prefill shape with position-correlated queries (recipe "local"), for the attention's packing.
+PREFILL_LOCAL_BF16 = Workload("prefill_local_bf16_B4_T8192_Hq16_Hkv4_d128_S64_k16_W512", B=4, T=8192, L=8192, Hq=16,
+                              Hkv=4, d=128, S=64, topk=16, W=512, dtype="bf16", recipe="local")
 TRAIN_BF16 = Workload("train_bf16_B2_T8192_Hq16_Hkv4_d128_S64_k16_W512", B=2, T=8192, L=8192, Hq=16, Hkv=4, d=128,
                       S=64, topk=16, W=512, dtype="bf16", recipe="scaled")
 
@@ -81,6 +87,18 @@ def _randn(shape, g, device) -> torch.Tensor:
     return torch.randn(*shape, generator=g, device=device, dtype=torch.float32)
 
 
+def _ar1_positions(e: torch.Tensor, rho: float) -> torch.Tensor:
+    """x_i = rho x_(i-1) + sqrt(1 - rho^2) e_i along dim 2 (x_0 = e_0), as
+    x_i = rho^i sum_(j<=i) rho^-j c_j e_j in float64 (c_0 = 1, c_j = sqrt(1 - rho^2))."""
+    T = e.shape[2]
+    j = torch.arange(T, device=e.device, dtype=torch.float64)
+    c = torch.full((T,), math.sqrt(1.0 - rho * rho), device=e.device, dtype=torch.float64)
+    c[0] = 1.0
+    wgt = (rho ** -j) * c
+    x = torch.cumsum(e.to(torch.float64) * wgt[None, None, :, None], dim=2) * (rho ** j)[None, None, :, None]
+    return x.to(torch.float32)
+
+
 def _qcal(q: torch.Tensor, d: int, g, device):
     """q^ = q + W_up (W_down q), rank 32, weights N(0, 1/128) (input recipe, upstream of the path).
     Returns (q^, W_down [32, d], W_up [d, 32])."""
@@ -91,7 +109,7 @@ def _qcal(q: torch.Tensor, d: int, g, device):
 
 def prefill_inputs(w: Workload, seed: int = 0, device="cpu", with_dout: bool = False) -> dict:
     """q, q_hat [B,Hq,T,d]; k, v [B,Hkv,L,d]; q_land [B,Hq,Nc,d]; optional dout [B,Hq,T,d]; with the
-    "scaled" recipe also the Q-Cal weights that made q_hat, w_down [32,d] and w_up [d,32]."""
+    "scaled" and "local" recipes also the Q-Cal weights that made q_hat, w_down [32,d] and w_up [d,32]."""
     g = _gen(seed, device)
     B, T, L, Hq, Hkv, d, Nc = w.B, w.T, w.L, w.Hq, w.Hkv, w.d, w.Nc
     if w.recipe == "tiny":
@@ -100,9 +118,12 @@ def prefill_inputs(w: Workload, seed: int = 0, device="cpu", with_dout: bool = F
         v = _randn((B, Hkv, L, d), g, device)
         q_land = _randn((B, Hq, Nc, d), g, device)
         q_hat = _randn((B, Hq, T, d), g, device)
-    elif w.recipe == "scaled":
+    elif w.recipe in ("scaled", "local"):
         s = d ** -0.25
-        q = _randn((B, Hq, T, d), g, device) * s
+        q = _randn((B, Hq, T, d), g, device)
+        if w.recipe == "local":
+            q = _ar1_positions(q, 0.995)
+        q = q * s
         k = _randn((B, Hkv, L, d), g, device) * s
         v = _randn((B, Hkv, L, d), g, device) * s
         q_land = _randn((B, Hq, Nc, d), g, device)
@@ -110,7 +131,7 @@ def prefill_inputs(w: Workload, seed: int = 0, device="cpu", with_dout: bool = F
     else:
         raise ValueError(f"prefill recipe {w.recipe!r}")
     out = {"q": q, "k": k, "v": v, "q_land": q_land, "q_hat": q_hat}
-    if w.recipe == "scaled":
+    if w.recipe in ("scaled", "local"):
         out.update(w_down=w_down, w_up=w_up)
     if with_dout:
         out["dout"] = _randn((B, Hq, T, d), g, device)
