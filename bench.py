@@ -625,8 +625,10 @@ def profile_case(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     st = args.profile
-    if st in ("summary", "decode"):
-        w = W.decode_sweep(524288) if st == "decode" else W.decode_sweep(131072)
+    if st in ("summary", "decode", "decode_multi"):
+        w = W.decode_sweep(524288) if st != "summary" else W.decode_sweep(131072)
+        if st == "decode_multi":
+            w = w.with_(name="decode_m4_bf16_B1_L524288", T=4, q_pos0=w.L - 4)
         x = W.decode_inputs(w, seed=2000, device=dev)
         k_sum, b_sum = H.chunk_summary(x["k_cache"], x["q_land"], w.S)
         if st == "summary":
@@ -670,7 +672,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="hils", choices=("hils", "reference"))
     ap.add_argument("--quick", action="store_true", help="headline only (no decode sweep / training blocks)")
-    ap.add_argument("--profile", choices=("summary", "select", "select_qcal", "attn", "decode", "bwd", "bsa"),
+    ap.add_argument("--profile",
+                    choices=("summary", "select", "select_qcal", "attn", "decode", "decode_multi", "bwd", "bsa"),
                     help="run --steps untimed launches of one stage for an ncu capture; no bench line")
     args = ap.parse_args()
     if args.profile:

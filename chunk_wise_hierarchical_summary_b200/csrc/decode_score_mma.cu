@@ -3,7 +3,7 @@
 // Right", Eq. 7) of M <= 8 queries against every candidate summary, with each summary row read from
 // HBM once for all M queries. bf16, d 128.
 //
-// Persistent kernel over units (b, head h, slice of 128 candidates), three CTAs per SM:
+// Persistent kernel over units (b, head h, slice of 128 candidates), two CTAs per SM:
 //   warp 4     producer: the slice's k' rows (TMA, two 64-column boxes, 128-byte swizzle) and the M query
 //              rows of the head (bulk copies into padded rows), into a kStages-deep ring.
 //   warps 0-3  warp w: rows 32w .. 32w+31 of the slice, as two m16 tiles of mma.sync m16n8k16 (k' rows as
@@ -26,7 +26,7 @@ namespace {
 constexpr int kStages = 3;
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
-constexpr int kCtasPerSm = 3;
+constexpr int kCtasPerSm = 2;  // shared memory (3 stages of 34 KB) holds two CTAs per SM: the grid stays resident
 constexpr int kRows = 128;                      // candidates per slice
 constexpr uint32_t kKBytes = kRows * 256;       // 128 rows x 128 columns bf16
 constexpr uint32_t kQRowBytes = 272;            // a query row (256 B) padded: conflict-free fragment reads
