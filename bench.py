@@ -206,8 +206,10 @@ ATTN_TC_TRAFFIC_BYTES = 241742336 + 102183680
 
 
 def base_config(w: W.Workload, world: int) -> dict:
+    """The workload both arms report (identical dicts, so the two lines name the same configuration)."""
     return {"workload": w.name, "global_batch": w.B * world, "seq_len": w.T,
-            "parallelism": f"dp{world} (independent sequences per GPU)"}
+            "parallelism": f"dp{world} (independent sequences per GPU)",
+            "l2": "flushed (256 MiB write) between timed prefill steps, outside the events"}
 
 
 # ----------------------------------------------------------------------------- algorithmic work
@@ -565,50 +567,60 @@ def oracle_prefill_sample(x_cpu, w: W.Workload, groups, row_blocks, block_rows, 
     return secs, rows_done * w.G / w.Hq, blocks_done
 
 
+ORACLE_BLOCKS, ORACLE_BLOCK_ROWS = 64, 128
+
+
+def oracle_sample_text(w: W.Workload, slices: int) -> str:
+    return (f"{slices} (batch, KV group) slice(s) of the prefill workload, each with all its {w.Nc} chunk summaries "
+            f"and {ORACLE_BLOCKS} evenly spaced blocks of {ORACLE_BLOCK_ROWS} query rows (all {w.G} heads); "
+            f"tokens counted as rows*G/Hq")
+
+
 def cpu_baseline(x_gpu, w, budget_s=15.0):
+    """The oracle as it stands on the host cores: whole (batch, KV group) slices (see oracle_sample_text)
+    until about `budget_s` seconds of CPU time are spent."""
     import oracle
 
     x_cpu = {n: x_gpu[n].cpu() for n in ("q", "k", "v", "q_hat", "q_land")}
     groups = [(b, g) for b in range(w.B) for g in range(w.Hkv)]
-    secs, tokens, blocks = 0.0, 0.0, 0
+    secs, tokens = 0.0, 0.0
     done = []
     for bg in groups:  # whole (batch, group) slices until the time budget is spent
-        s, t, nb = oracle_prefill_sample(x_cpu, w, [bg], 64, 128)
-        secs, tokens, blocks = secs + s, tokens + t, blocks + nb
+        s, t, _ = oracle_prefill_sample(x_cpu, w, [bg], ORACLE_BLOCKS, ORACLE_BLOCK_ROWS)
+        secs, tokens = secs + s, tokens + t
         done.append(bg)
         if secs > budget_s:
             break
     return {"value": tokens / secs, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
-            "sample": f"{len(done)} of {len(groups)} (batch, KV group) slices, each with all its {w.Nc} chunk "
-                      f"summaries and 64 evenly spaced blocks of 128 query rows (all {w.G} heads); tokens counted "
-                      f"as rows*G/Hq; {secs:.1f} s of CPU time"}
+            "sample": oracle_sample_text(w, len(done)) + f"; {secs:.1f} s of CPU time"}
 
 
 def run_reference(args, dist):
-    """Reference arm: the fp64 CPU oracle on a bounded sample of the prefill workload, per step."""
+    """Reference arm: the fp64 CPU oracle on the host cores, one step = the same sample unit as the
+    cpu_baseline leg (one whole (batch, KV group) slice), the slices visited in turn. Under torchrun only
+    rank 0 runs it; the other ranks exit without work."""
     if dist.rank != 0:
         return
     import oracle
 
     w = W.PREFILL_BF16
     x = W.prefill_inputs(w, seed=1000, device="cpu")
-    groups, blocks, rows = [(0, 0)], 2, 32
-    for _ in range(args.warmup):
-        oracle_prefill_sample(x, w, groups, blocks, rows)
+    groups = [(b, g) for b in range(w.B) for g in range(w.Hkv)]
+    for n in range(args.warmup):
+        oracle_prefill_sample(x, w, [groups[n % len(groups)]], ORACLE_BLOCKS, ORACLE_BLOCK_ROWS)
     total, tokens = 0.0, 0.0
-    for _ in range(args.steps):
-        s, t, _ = oracle_prefill_sample(x, w, groups, blocks, rows)
+    for n in range(args.steps):
+        s, t, _ = oracle_prefill_sample(x, w, [groups[n % len(groups)]], ORACLE_BLOCKS, ORACLE_BLOCK_ROWS)
         total += s
         tokens += t
     value = tokens / total
-    sample = (f"1 (batch, KV group) slice x {blocks} blocks of {rows} query rows per step; tokens = rows*G/Hq")
     line = {"metric": METRIC, "value": value,
             "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": base_config(w, 1),
+            "config": base_config(w, args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
-                             "sample": sample},
+                             "sample": oracle_sample_text(w, 1) + " per step"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
 
@@ -665,6 +677,23 @@ def profile_case(args):
 
 # ----------------------------------------------------------------------------- main
 
+def decode_summary(decode: dict, extra: dict) -> dict:
+    """The decode half of the headline in a few fields: us/token and the HBM fraction at the decode
+    workload, then the sweep's (L, us/token, HBM fraction) and multi-token decode, when run."""
+    out = {"workload": decode["workload"], "us_per_token": decode["us_per_token"],
+           "hbm_frac": decode["roofline"]["frac"], "achieved_gbs": decode["roofline"]["achieved"],
+           "peak_gbs": decode["roofline"]["peak"], "bytes_per_step": decode["bytes_per_step"]["total"],
+           "l2": "not flushed: one fixed query per sequence replayed, 629 MB touched per step (5x L2)"}
+    if "decode_sweep" in extra:
+        out["sweep_L_us_frac"] = [[r["L"], round(r["us_per_token"], 2), round(r["hbm_frac"], 4)]
+                                  for r in extra["decode_sweep"]]
+    if "decode_multi" in extra:
+        m = extra["decode_multi"]
+        out["multi_m4_us_per_step"] = m["us_per_step"]
+        out["multi_m4_hbm_frac"] = m["roofline"]["frac"]
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -716,14 +745,13 @@ def main():
         if dist.world == 1:
             cpu = cpu_baseline(pre["x"], w)
         launches = pre["launches_per_step"] * args.steps
+        pre["roofline"]["peak_source"] = peak_src
         line = {
             "metric": METRIC,
             "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {**base_config(w, dist.world),
-                       "l2": "flushed (256 MiB write) between timed steps, outside the events",
-                       "peaks": peak_src},
+            "config": base_config(w, dist.world),
             "stage_ms": {"chunk_summary": pre["stage_ms"][0], "select_topk": pre["stage_ms"][1],
                          "attn_fwd": pre["stage_ms"][2]},
             "roofline": pre["roofline"],
@@ -732,8 +760,10 @@ def main():
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": pre["clocks"],
-            "decode": decode,
             **extra,
+            "decode_detail": decode,
+            # last, so that the headline's decode half is in any tail of the line
+            "decode": decode_summary(decode, extra),
         }
         if dist.rank == 0:
             print(json.dumps(line, default=lambda o: getattr(o, "name", str(o))))

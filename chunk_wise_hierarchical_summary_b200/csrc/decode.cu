@@ -956,7 +956,7 @@ cudaError_t launch_t(const Dims &D, const void *q, const void *q_hat, const void
     unsigned int *selcount = (unsigned int *)(w + P.off_selcount);
     // One CTA per (b, KV group, query) selects the top-k of a whole candidate list. With few groups and a
     // long list (a few sequences over a cache of a million tokens or more) that leaves most SMs idle: the
-    // list is then split over ceil(n / 1024) CTAs per group whose top-(k+1) lists the last CTA merges.
+    // list is then split over ceil(n / 1024) CTAs per group whose top-k lists the last CTA merges.
     // (Measured at B1: 8184 candidates faster on one CTA, 16376 and more faster split.)
     const bool wide = D.T == 1 && D.B * D.Hkv < 32 && P.n >= 12288 && next_pow2(P.nparts * D.topk) <= kSelMerge;
     cudaError_t es;

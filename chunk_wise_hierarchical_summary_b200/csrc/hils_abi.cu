@@ -36,6 +36,8 @@ cudaError_t launch_select_tc_qcal(const Dims &D, const void *q, const void *w_do
 int bsa_max_candidates(const Dims &D);
 cudaError_t launch_bsa_select_topk(const Dims &D, int dtype, const void *q, const void *k, int *idx, float *gap,
                                    float *mass, cudaStream_t stream);
+unsigned int wait_expiry_error_flags(bool clear);
+cudaError_t launch_wait_expiry(uint32_t max_polls, int arrive_first, cudaStream_t stream);
 
 namespace {
 
@@ -123,6 +125,9 @@ hils_status check_device_errors() {
     if (decode_error_flags(true) != 0)
         return fail(HILS_ERR_TIMEOUT, "hils_check: a decode tile's bulk copy did not complete within its wait "
                     "budget; that call's output is invalid");
+    if (wait_expiry_error_flags(true) != 0)
+        return fail(HILS_ERR_TIMEOUT, "hils_check: the test hook's bounded wait expired (nothing arrived at its "
+                    "barrier)");
     return HILS_OK;
 }
 
@@ -361,6 +366,14 @@ hils_status hils_attn_bwd(const hils_params *p, const void *q, const void *k, co
     return cuda_status(launch_attn_bwd(D, p->dtype, q, k, v, q_hat, q_land, k_sum, b_sum, idx, out, lse, dout, dq, dk,
                                        dv, dq_hat, dq_land, workspace, (cudaStream_t)stream),
                        fn);
+}
+
+hils_status hils_test_wait_expiry(uint32_t max_polls, int32_t arrive_first, hils_stream_t stream) {
+    const char *fn = "hils_test_wait_expiry";
+    if (max_polls < 1 || max_polls > HILS_TEST_WAIT_MAX_POLLS)
+        return fail(HILS_ERR_INVALID_ARG, "%s: max_polls=%u outside [1, %u]", fn, max_polls,
+                    (unsigned)HILS_TEST_WAIT_MAX_POLLS);
+    return cuda_status(launch_wait_expiry(max_polls, arrive_first != 0, (cudaStream_t)stream), fn);
 }
 
 hils_status hils_check(hils_stream_t stream) {

@@ -42,11 +42,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Returns false if the phase did not complete within the poll budget.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kMaxWaitPolls; ++i)
+// Returns false if the phase did not complete within `max_polls` polls.
+__device__ __forceinline__ bool mbar_wait_polls(uint64_t *bar, uint32_t parity, uint32_t max_polls) {
+    for (uint32_t i = 0; i < max_polls; ++i)
         if (mbar_try_wait(bar, parity)) return true;
     return false;
+}
+
+// The wait every kernel of the library uses: false if the phase did not complete within kMaxWaitPolls.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+    return mbar_wait_polls(bar, parity, kMaxWaitPolls);
 }
 
 // 1-D bulk copy global -> shared (this CTA), completing `bytes` of transaction on `bar`.

@@ -28,7 +28,7 @@ OP_SUMMARY, OP_SELECT, OP_ATTN_FWD, OP_DECODE, OP_ATTN_BWD = 0, 1, 2, 3, 4
 # Every symbol include/hils.h declares (checked by the tests against the header and the library).
 EXPORTED = ("hils_workspace_size", "hils_chunk_summary", "hils_chunk_summary_shared_query", "hils_select_topk",
             "hils_select_topk_qcal", "hils_bsa_select_topk", "hils_attn_fwd", "hils_decode", "hils_attn_bwd", "hils_check", "hils_status_string", "hils_last_error",
-            "hils_version", "hils_decode_noalloc")
+            "hils_version", "hils_decode_noalloc", "hils_test_wait_expiry")
 
 
 class HilsError(RuntimeError):
@@ -68,6 +68,8 @@ def _load() -> ctypes.CDLL:
     lib.hils_attn_bwd.restype = st
     lib.hils_decode_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.hils_decode_noalloc.restype = st
+    lib.hils_test_wait_expiry.argtypes = [ctypes.c_uint32, ctypes.c_int32, vp]
+    lib.hils_test_wait_expiry.restype = st
     lib.hils_check.argtypes = [vp]
     lib.hils_check.restype = st
     lib.hils_status_string.argtypes = [st]

@@ -212,7 +212,9 @@ HILS_API hils_status hils_attn_bwd(const hils_params *p, const void *q, const vo
  *  - Sizes whose decode workspace (hils_workspace_size(p, HILS_OP_DECODE)) exceeds the array are
  *    rejected with HILS_ERR_UNSUPPORTED before anything is enqueued.
  *  - The first call on a device (with that device current) looks up the array's device address
- *    with cudaGetSymbolAddress; make that first call before any stream capture. Later calls reuse it.
+ *    with cudaGetSymbolAddress; make that first call before any stream capture. Later calls reuse it
+ *    for the life of the process, so a cudaDeviceReset (or anything else that destroys the device's
+ *    primary context) invalidates it: do not call this entry point on that device afterwards.
  *  - All calls on a device share the one array and it keeps the previous call's contents: calls
  *    whose GPU work overlaps (e.g. on two streams without ordering between them) race and corrupt
  *    each other's results; order them on one stream or with events. Every scratch byte a call reads
@@ -224,6 +226,20 @@ HILS_API hils_status hils_decode_noalloc(const hils_params *p, const void *q, co
                                          const void *k_cache, const void *v_cache, const void *k_sum,
                                          const float *b_sum, void *out, float *lse, int32_t *idx_out,
                                          hils_stream_t stream);
+
+/*
+ * Test hook of the failure detection; the paper has no counterpart. Every kernel of this library waits on
+ * its copies and tensor-core operations with a bounded mbarrier wait; when a wait runs out the kernel
+ * records it in a device error word and leaves, and the next hils_check returns HILS_ERR_TIMEOUT. This call
+ * runs that same wait in one CTA on a barrier that nothing arrives at (arrive_first = 0), with a limit of
+ * max_polls polls (1 .. HILS_TEST_WAIT_MAX_POLLS), so the wait expires and is
+ * recorded; with arrive_first != 0 the CTA arrives first and the wait completes (a control). The barrier
+ * is fed by no copy and no tensor-core operation, so nothing is left in flight and the context stays
+ * usable. Returns after enqueueing; the outcome is read with hils_check. HILS_ERR_INVALID_ARG for a
+ * max_polls outside the range.
+ */
+#define HILS_TEST_WAIT_MAX_POLLS (1u << 20)
+HILS_API hils_status hils_test_wait_expiry(uint32_t max_polls, int32_t arrive_first, hils_stream_t stream);
 
 /* Waits for `stream`, then reports a device-side error word (HILS_ERR_TIMEOUT) or a CUDA error. */
 HILS_API hils_status hils_check(hils_stream_t stream);

@@ -52,3 +52,34 @@ def test_both_arms_share_metric_and_base_config():
     c1, c2 = bench.base_config(w, 1), bench.base_config(w, 4)
     assert c1["workload"] == c2["workload"] == w.name and c2["global_batch"] == 4 * c1["global_batch"]
     assert "TC/HBM roofline" in bench.METRIC
+
+
+def test_decode_summary_carries_the_headline_decode_half():
+    """The line's last key holds the decode workload's us/token and HBM fraction (and the sweep's), in a
+    few hundred characters, so any tail of the line shows them."""
+    import json
+
+    dec = {"workload": "decode_bf16_B8_L524288", "us_per_token": 129.0, "bytes_per_step": {"total": 628_800_000},
+           "roofline": {"frac": 0.75, "achieved": 4870.0, "peak": 6452.5}}
+    extra = {"decode_sweep": [{"L": L, "us_per_token": 30.0 + L / 1e5, "hbm_frac": 0.1} for L in W.DECODE_SWEEP_L],
+             "decode_multi": {"us_per_step": 192.0, "roofline": {"frac": 0.6}}}
+    s = bench.decode_summary(dec, extra)
+    assert s["us_per_token"] == 129.0 and s["hbm_frac"] == 0.75
+    assert [r[0] for r in s["sweep_L_us_frac"]] == list(W.DECODE_SWEEP_L)
+    assert len(json.dumps(s)) < 800
+    assert "sweep_L_us_frac" not in bench.decode_summary(dec, {})
+
+
+def test_reference_arm_line_matches_the_gpu_arms_config_and_sample(capsys):
+    """--impl reference prints one line whose metric and config are the GPU arm's, and whose cpu_baseline
+    sample is the unit the GPU arm's cpu_baseline leg times (one whole (batch, KV group) slice)."""
+    import argparse
+    import json
+
+    args = argparse.Namespace(gpus=1, steps=1, warmup=0)
+    bench.run_reference(args, bench.Dist(1))
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["config"] == bench.base_config(W.PREFILL_BF16, 1)
+    assert line["cpu_baseline"]["sample"].startswith(bench.oracle_sample_text(W.PREFILL_BF16, 1))
+    assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
