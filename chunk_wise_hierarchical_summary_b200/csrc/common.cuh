@@ -84,6 +84,47 @@ __device__ __forceinline__ void block_bitonic_sort(uint64_t *keys, int n) {
     __syncthreads();
 }
 
+// Ascending bitonic sort of 32*NPL 64-bit keys held in registers by one warp; element e of the
+// sequence is v[e % NPL] of lane e / NPL. No shared memory, no barriers.
+template <int NPL>
+__device__ __forceinline__ void warp_bitonic_sort(uint64_t (&v)[NPL]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int size = 2; size <= 32 * NPL; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            if (stride >= NPL) {
+                const int ls = stride / NPL;
+                const bool lower = (lane & ls) == 0;
+#pragma unroll
+                for (int i = 0; i < NPL; ++i) {
+                    const int e = lane * NPL + i;
+                    const bool up = (e & size) == 0;
+                    const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v[i], ls);
+                    const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v[i] >> 32), ls);
+                    const uint64_t p = ((uint64_t)hi << 32) | lo;
+                    const bool keep_min = (lower == up);
+                    v[i] = keep_min ? (v[i] < p ? v[i] : p) : (v[i] > p ? v[i] : p);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < NPL; ++i) {
+                    const int j = i ^ stride;
+                    if (j > i) {
+                        const int e = lane * NPL + i;
+                        const bool up = (e & size) == 0;
+                        if ((v[i] > v[j]) == up) {
+                            const uint64_t t = v[i];
+                            v[i] = v[j];
+                            v[j] = t;
+                        }
+                    }
+                }
+            }
+        }
+    }
+}
+
 // Programmatic dependent launch: a kernel launched with launch_pdl may start while the grid before it
 // on the stream is still running; grid_dep_wait() blocks until that grid has completed and its memory
 // is visible (a no-op for an ordinary launch). Every CTA of such a kernel calls it before reading what

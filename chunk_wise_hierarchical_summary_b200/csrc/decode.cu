@@ -262,47 +262,6 @@ decode_score_kernel(Dims D, DecodePlan P, const T *__restrict__ q_hat, const T *
 
 // ---------------------------------------------------------------------------- 2. select
 
-// Ascending bitonic sort of 32*NPL 64-bit keys held in registers by one warp; element e of the
-// sequence is v[e % NPL] of lane e / NPL. No shared memory, no barriers.
-template <int NPL>
-__device__ __forceinline__ void warp_bitonic_sort(uint64_t (&v)[NPL]) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int size = 2; size <= 32 * NPL; size <<= 1) {
-#pragma unroll
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            if (stride >= NPL) {
-                const int ls = stride / NPL;
-                const bool lower = (lane & ls) == 0;
-#pragma unroll
-                for (int i = 0; i < NPL; ++i) {
-                    const int e = lane * NPL + i;
-                    const bool up = (e & size) == 0;
-                    const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v[i], ls);
-                    const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v[i] >> 32), ls);
-                    const uint64_t p = ((uint64_t)hi << 32) | lo;
-                    const bool keep_min = (lower == up);
-                    v[i] = keep_min ? (v[i] < p ? v[i] : p) : (v[i] > p ? v[i] : p);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < NPL; ++i) {
-                    const int j = i ^ stride;
-                    if (j > i) {
-                        const int e = lane * NPL + i;
-                        const bool up = (e & size) == 0;
-                        if ((v[i] > v[j]) == up) {
-                            const uint64_t t = v[i];
-                            v[i] = v[j];
-                            v[j] = t;
-                        }
-                    }
-                }
-            }
-        }
-    }
-}
-
 // Grid (parts, Hkv, B): each CTA owns kSelPart candidates of one group. It folds the per-head score
 // partials into LSE_h, forms 64-bit keys (group score desc, chunk id asc; all distinct), keeps its
 // local top-k by a shared-memory bitonic sort and writes them to the workspace. The last CTA of the

@@ -205,34 +205,50 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
 
     if (GATHER) {
-        // Gather mode: row (query) r of head j reads its caller-given ids, keeps the valid distinct
-        // ones ascending and writes them with their retrieval scores s^ = tau D + b' to the workspace.
-        if (j < G) {  // warp-uniform: every lane executes the TMEM loads
-            const int hh = j, K = D.topk;
-            const bool valid = i < D.T;
-            int cl[32];
-            int ns = 0;
+        // Gather mode: the caller-given ids of row (query) r are canonicalised once per row (valid ones,
+        // distinct, ascending: a 128-bit set in registers, candidates being < 128 here) into shared
+        // memory; then each head's warp writes their retrieval scores s^ = tau D + b' to the workspace.
+        // The operand stages are dead once every MMA has completed: [0, 66 KiB) holds the per-thread
+        // 33-float rows below, the canonical lists follow.
+        int *clist = reinterpret_cast<int *>(base + (size_t)kThreads * 33 * sizeof(float));
+        int *ccount = clist + kRows * D.topk;
+        const int K = D.topk;
+        const bool valid = i < D.T;
+        if (j == 0) {
+            uint32_t m0 = 0u, m1 = 0u, m2 = 0u, m3 = 0u;
             if (valid) {
                 const int *src = idx + (((size_t)b * D.Hkv + g) * D.T + i) * K;
                 for (int t = 0; t < K; ++t) {
                     const int c = src[t];
                     if (c < 0 || c >= n_r) continue;
-                    bool dup = false;
-                    for (int u = 0; u < ns; ++u) dup |= (cl[u] == c);
-                    if (dup) continue;
-                    int pos = ns;
-                    while (pos > 0 && cl[pos - 1] > c) {
-                        cl[pos] = cl[pos - 1];
-                        --pos;
-                    }
-                    cl[pos] = c;
-                    ++ns;
+                    const uint32_t bit = 1u << (c & 31);
+                    const int w = c >> 5;
+                    m0 |= (w == 0) ? bit : 0u;
+                    m1 |= (w == 1) ? bit : 0u;
+                    m2 |= (w == 2) ? bit : 0u;
+                    m3 |= (w == 3) ? bit : 0u;
                 }
             }
+            int ns = 0;
+            const uint32_t words[4] = {m0, m1, m2, m3};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                uint32_t x = words[w];
+                while (x) {
+                    clist[r * K + ns++] = 32 * w + __ffs(x) - 1;
+                    x &= x - 1u;
+                }
+            }
+            ccount[r] = ns;
+        }
+        __syncthreads();
+        if (j < G) {  // warp-uniform: every lane executes the TMEM loads
+            const int hh = j;
+            const int ns = ccount[r];
+            const int *cl = clist + r * K;
             float *dst_s = ws_shat + (((size_t)b * D.Hq + g * G + hh) * D.T + i) * K;
-            // The operand stages are dead once every MMA has completed: each thread copies a 32-column
-            // block of its row into a private shared-memory row (stride 33 floats, conflict-free) and
-            // reads the selected columns back by index.
+            // each thread copies a 32-column block of its row into a private shared-memory row (stride 33
+            // floats, conflict-free) and reads the selected columns back by index
             float *row32 = reinterpret_cast<float *>(base) + (size_t)tid * 33;
             int u = 0;
 #pragma unroll 1
