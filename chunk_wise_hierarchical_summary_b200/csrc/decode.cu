@@ -1,7 +1,7 @@
 // Single-token decode over a long KV cache: stages (b)-(d) for one query at position L-1
 // ("Hierarchical Sparse Attention Done Right", Eq. 7, Sec. 3 RQ1, Sec. 4 "GQA", Eq. 10).
 //
-// Three launches (plus one memset of the counters):
+// Three launches (the score grid also clears the two counter arrays the later grids count with):
 //  1. score    persistent, one CTA per SM: a producer lane keeps a ring of bulk copies of 128-candidate
 //              summary slices (32 KiB at d 128 bf16) in flight; consumer warps compute
 //              s^_{h,c} = tau q^_h . k'_{h,c} + b'_{h,c} into a score buffer plus per-warp partials
@@ -31,7 +31,8 @@ cudaError_t launch_decode_attn_mma(const Dims &D, int n, int ntiles, const void 
 unsigned int decode_attn_mma_error_flags(bool clear);
 bool decode_score_mma_supported(const Dims &D, int dtype, const void *q_hat, const void *k_sum);
 cudaError_t launch_decode_score_mma(const Dims &D, int n, int nslices, const void *q_hat, const void *k_sum,
-                                    const float *b_sum, float *scores, float *part, cudaStream_t stream);
+                                    const float *b_sum, float *scores, float *part, unsigned int *clear, int nclear,
+                                    cudaStream_t stream);
 unsigned int decode_score_mma_error_flags(bool clear);
 
 namespace {
@@ -111,7 +112,8 @@ struct ScoreCfg {
 template <typename T>
 __global__ void __launch_bounds__(ScoreCfg<T>::kThreads)
 decode_score_kernel(Dims D, DecodePlan P, const T *__restrict__ q_hat, const T *__restrict__ k_sum,
-                    const float *__restrict__ b_sum, float *__restrict__ scores, float *__restrict__ part) {
+                    const float *__restrict__ b_sum, float *__restrict__ scores, float *__restrict__ part,
+                    unsigned int *__restrict__ clear, int nclear) {
     using C = ScoreCfg<T>;
     constexpr int NS = C::kStages, WPS = C::kWarpsPerSlot;
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -121,6 +123,10 @@ decode_score_kernel(Dims D, DecodePlan P, const T *__restrict__ q_hat, const T *
     const size_t slot_bytes = (size_t)P.per * d * sizeof(T);
     const int units = D.B * D.Hq * P.nslices;
     grid_dep_launch();  // the selection's CTAs may take SMs as this grid's CTAs finish
+    // The later grids' counters start at zero: they read them only after this grid has completed (the
+    // selection's griddepcontrol.wait or an ordinary launch; the attention through the selection's).
+    if (blockIdx.x == 0)
+        for (int i = tid; i < nclear; i += blockDim.x) clear[i] = 0u;
     if (tid == 0) {
         for (int i = 0; i < NS; ++i) {
             mbar_init(&full[i], 1);
@@ -893,11 +899,16 @@ cudaError_t launch_t(const Dims &D, const void *q, const void *q_hat, const void
     int *sel = (int *)(w + P.off_sel);
     float *partial = (float *)(w + P.off_attn);
     unsigned int *counters = (unsigned int *)(w + P.off_count);
-    // Both counter arrays (attention, selection) are adjacent: clear them in one call.
-    cudaError_t e = cudaMemsetAsync(counters, 0, P.total - P.off_count, stream);
-    if (e != cudaSuccess) return e;
+    // Both counter arrays (attention, selection) are adjacent; the score grid clears them, and without
+    // candidates (no score grid) one memset does.
+    const int nclear = (int)((P.total - P.off_count) / sizeof(unsigned int));
+    if (P.n == 0) {
+        cudaError_t e = cudaMemsetAsync(counters, 0, P.total - P.off_count, stream);
+        if (e != cudaSuccess) return e;
+    }
     if (P.n > 0 && D.T > 1) {
-        cudaError_t es = launch_decode_score_mma(D, P.n, P.nslices, q_hat, k_sum, b_sum, scores, part, stream);
+        cudaError_t es = launch_decode_score_mma(D, P.n, P.nslices, q_hat, k_sum, b_sum, scores, part, counters,
+                                                 nclear, stream);
         if (es != cudaSuccess) return es;
     } else if (P.n > 0) {
         using C = ScoreCfg<T>;
@@ -910,7 +921,7 @@ cudaError_t launch_t(const Dims &D, const void *q, const void *q_hat, const void
         const int sms = num_sms();
         const int grid = units < sms ? units : sms;
         k1<<<grid, ScoreCfg<T>::kThreads, smem1, stream>>>(D, P, (const T *)q_hat, (const T *)k_sum, b_sum, scores,
-                                                           part);
+                                                           part, counters, nclear);
     }
     unsigned int *selcount = (unsigned int *)(w + P.off_selcount);
     // One CTA per (b, KV group, query) selects the top-k of a whole candidate list. With few groups and a

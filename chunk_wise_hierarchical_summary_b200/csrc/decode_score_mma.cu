@@ -38,7 +38,8 @@ __device__ unsigned int g_score_mma_errors = 0;
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 decode_score_mma_kernel(const __grid_constant__ CUtensorMap kmap, Dims D, int n, int nslices,
                         const __nv_bfloat16 *__restrict__ q_hat, const float *__restrict__ b_sum,
-                        float *__restrict__ scores, float *__restrict__ part) {
+                        float *__restrict__ scores, float *__restrict__ part, unsigned int *__restrict__ clear,
+                        int nclear) {
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
     unsigned char *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -46,6 +47,9 @@ decode_score_mma_kernel(const __grid_constant__ CUtensorMap kmap, Dims D, int n,
     const int M = D.T;
     const long long units = (long long)D.B * D.Hq * nslices;
     grid_dep_launch();  // the selection's CTAs may take SMs as this grid's CTAs finish
+    // the later grids' counters start at zero (they read them only after this grid has completed)
+    if (blockIdx.x == 0)
+        for (int i = tid; i < nclear; i += blockDim.x) clear[i] = 0u;
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
@@ -199,7 +203,8 @@ unsigned int decode_score_mma_error_flags(bool clear) {
 
 // scores [B, Hq, M, n] fp32; part [B, Hq, M, nslices, 4 warps, (max, sum)] fp32; slices of 128 candidates.
 cudaError_t launch_decode_score_mma(const Dims &D, int n, int nslices, const void *q_hat, const void *k_sum,
-                                    const float *b_sum, float *scores, float *part, cudaStream_t stream) {
+                                    const float *b_sum, float *scores, float *part, unsigned int *clear, int nclear,
+                                    cudaStream_t stream) {
     CUtensorMap kmap;
     if (!make_tmap_bf16_2d(&kmap, k_sum, (uint64_t)D.B * D.Hq * D.Nc, 128, 128, kRows)) return cudaErrorInvalidValue;
     const size_t smem = 1024 + kStages * (kKBytes + kQBytes);
@@ -207,7 +212,7 @@ cudaError_t launch_decode_score_mma(const Dims &D, int n, int nslices, const voi
     const long long units = (long long)D.B * D.Hq * nslices;
     const int grid = (int)std::min<long long>(units, (long long)kCtasPerSm * num_sms());
     decode_score_mma_kernel<<<grid, kThreads, smem, stream>>>(kmap, D, n, nslices, (const __nv_bfloat16 *)q_hat,
-                                                             b_sum, scores, part);
+                                                             b_sum, scores, part, clear, nclear);
     return cudaGetLastError();
 }
 
