@@ -537,6 +537,8 @@ decode_select_warp_kernel(Dims D, DecodePlan P, const float *__restrict__ scores
     const int G = D.G, K = D.topk;
     const int n = window_left(D.q_pos0 + m, D.W, D.S) / D.S;
     const size_t bgm = ((size_t)b * D.Hkv + g) * M + m;
+    // the attention grid may start now: its CTAs load and fold their window tiles while this grid selects
+    grid_dep_launch();
     grid_dep_wait();  // the score grid's scores and partials
     const size_t hs = (size_t)M * P.n;  // stride between the group's heads in the score rows
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = kSelWThreads / 32;

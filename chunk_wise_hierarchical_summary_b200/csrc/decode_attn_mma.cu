@@ -3,8 +3,9 @@
 // Sec. 3 RQ2, Eq. 10; Sec. 4 "GQA": the group's heads share every gathered tile).
 //
 // grid (nsplit, Hkv, B * M) for M = T query tokens per sequence (M > 1: multi-token decode): the tiles of
-// one (b, KV group, query) - its selected chunks, then its window tiles - are dealt round-robin to
-// nsplit CTAs. Per CTA:
+// one (b, KV group, query) - its window tiles, then its selected chunks - are dealt round-robin to
+// nsplit CTAs. A CTA's window tiles depend on no earlier grid, so they are loaded and folded into its
+// running softmax before griddepcontrol.wait, while the selection grid still runs. Per CTA:
 //   warp 4     producer: K and V tiles (TMA, 128-byte swizzle) into a kStages-deep ring.
 //   warps 0-3  per tile, on the warp-level tensor-core instruction (mma.sync m16n8k16, bf16 in, fp32
 //              accumulate) with the group's heads as the 8-wide N side:
@@ -69,8 +70,7 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     const size_t bgm = bg * M + m;            // this query's ids and counter
     const int pos = D.q_pos0 + m;
     const int l = window_left(pos, D.W, S);
-    grid_dep_wait();  // the selection grid's ids (and, through it, the scores)
-
+    const int wt = ntiles - K;  // window tiles of the sequence; the selected chunks follow them
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
@@ -78,20 +78,12 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
         }
         fence_mbar_init();
         int nt = 0;
-        for (int t = split; t < ntiles && nt < kMaxTiles; t += nsplit) {
+        for (int t = split; t < wt && nt < kMaxTiles; t += nsplit) {
             Tile tl;
-            if (t < K) {
-                const int c = sel[bgm * K + t];
-                if (c < 0) continue;
-                tl.j0 = c * S;
-                tl.jn = S;
-                tl.c = c;
-            } else {
-                tl.j0 = l + (t - K) * S;
-                tl.jn = min(S, pos + 1 - tl.j0);
-                tl.c = -1;
-                if (tl.jn <= 0) continue;
-            }
+            tl.j0 = l + t * S;
+            tl.jn = min(S, pos + 1 - tl.j0);
+            tl.c = -1;
+            if (tl.jn <= 0) continue;
             tiles[nt++] = tl;
         }
         s_nt = nt;
@@ -102,7 +94,8 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
             *reinterpret_cast<const uint4 *>(q + (((size_t)b * D.Hq + g * G + h) * M + m) * 128 + ch * 8);
     }
     __syncthreads();
-    const int nt = s_nt;
+    const int nw = s_nt;  // this CTA's window tiles: the head of its list
+    int nt = nw;
     bool ok = true;
 
     // running state of the consumer threads for heads 2*t4 and 2*t4+1 (log2 units)
@@ -110,25 +103,53 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     float o[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     const int g8 = lane >> 2, t4 = lane & 3;
 
+    // The selected chunks of this CTA, appended once the selection grid has completed.
+    auto append_selected = [&]() {
+        grid_dep_wait();  // the selection grid's ids (and, through it, the scores)
+        __syncthreads();  // every thread is past its pre-wait tiles before the list grows
+        if (tid == 0) {
+            int n2 = nw;
+            for (int t = split + ((wt - split + nsplit - 1) / nsplit) * nsplit; t < ntiles && n2 < kMaxTiles;
+                 t += nsplit) {
+                if (t < wt) continue;
+                const int c = sel[bgm * K + (t - wt)];
+                if (c < 0) continue;
+                Tile tl;
+                tl.j0 = c * S;
+                tl.jn = S;
+                tl.c = c;
+                tiles[n2++] = tl;
+            }
+            s_nt = n2;
+        }
+        __syncthreads();
+        nt = s_nt;
+    };
+
     if (warp == kConsumerWarps) {
         // ---------------------------------------------------------------- producer
-        if (lane == 0) {
-            for (int i = 0; i < nt; ++i) {
-                const int st = i % kStages;
-                if (i >= kStages && !mbar_wait_bounded(&empty[st], ((i / kStages) - 1) & 1)) {
-                    ok = false;
-                    break;
+        auto produce = [&](int i0, int i1) {
+            if (lane == 0) {
+                for (int i = i0; i < i1 && ok; ++i) {
+                    const int st = i % kStages;
+                    if (i >= kStages && !mbar_wait_bounded(&empty[st], ((i / kStages) - 1) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    unsigned char *Kt = base + st * 2 * kTileBytes;
+                    const int y = (int)(bg * D.L) + tiles[i].j0;
+                    mbar_arrive_expect_tx(&full[st], 2 * kTileBytes);
+                    tma_load_2d(Kt, &kmap, 0, y, &full[st]);
+                    tma_load_2d(Kt + 8192, &kmap, 64, y, &full[st]);
+                    tma_load_2d(Kt + kTileBytes, &vmap, 0, y, &full[st]);
+                    tma_load_2d(Kt + kTileBytes + 8192, &vmap, 64, y, &full[st]);
                 }
-                unsigned char *Kt = base + st * 2 * kTileBytes;
-                const int y = (int)(bg * D.L) + tiles[i].j0;
-                mbar_arrive_expect_tx(&full[st], 2 * kTileBytes);
-                tma_load_2d(Kt, &kmap, 0, y, &full[st]);
-                tma_load_2d(Kt + 8192, &kmap, 64, y, &full[st]);
-                tma_load_2d(Kt + kTileBytes, &vmap, 0, y, &full[st]);
-                tma_load_2d(Kt + kTileBytes + 8192, &vmap, 64, y, &full[st]);
             }
-        }
-        __syncwarp();
+            __syncwarp();
+        };
+        produce(0, nw);
+        append_selected();
+        produce(nw, nt);
     } else {
         // ---------------------------------------------------------------- consumers
         const int mi = lane >> 3, r8 = lane & 7;
@@ -136,7 +157,8 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
         const float sc2 = D.tau * kLog2e;
         // query rows (b, head, m) of [B, Hq, M, ...]: head h of the group at hrow0 + h * M
         const size_t hrow0 = ((size_t)b * D.Hq + g * G) * M + m;
-        for (int i = 0; i < nt; ++i) {
+        auto consume = [&](int i0, int i1) {
+          for (int i = i0; i < i1; ++i) {
             const int st = i % kStages;
             const Tile tl = tiles[i];
             // the chunk's retrieval score for this thread's two heads, fetched before the tile wait
@@ -245,7 +267,11 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
-        }
+          }
+        };
+        consume(0, nw);
+        append_selected();
+        if (ok) consume(nw, nt);
         // this CTA's partial per head: (M, l, -, -) then o[128], laid out [B*Hq][nsplit][kPartStride]
         if (ok) {
 #pragma unroll

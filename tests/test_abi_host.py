@@ -154,3 +154,10 @@ def test_select_too_many_chunks_for_one_cta():
     p = P(T=1, L=1 << 20, q_pos0=(1 << 20) - 1)
     st = H.lib.hils_select_topk(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, None, 0, None)
     assert st == 2 and b"hils_decode" in H.lib.hils_last_error()
+
+
+def test_wait_expiry_hook_rejects_limits_before_any_launch():
+    """The failure-detection test hook validates its poll limit on the host (no CUDA call is made)."""
+    assert H.lib.hils_test_wait_expiry(0, 0, None) == H.HilsError(1, "").status
+    assert H.lib.hils_test_wait_expiry((1 << 20) + 1, 1, None) == 1
+    assert b"max_polls" in H.lib.hils_last_error()
