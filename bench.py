@@ -272,20 +272,18 @@ def bench_prefill(args, dist, dev, H, peaks):
     k_sum = torch.empty((w.B, w.Hq, w.Nc, w.d), dtype=torch.bfloat16, device=dev)
     b_sum = torch.empty((w.B, w.Hq, w.Nc), dtype=torch.float32, device=dev)
     idx = torch.empty((w.B, w.Hkv, w.T, w.topk), dtype=torch.int32, device=dev)
+    shat = torch.empty((w.B, w.Hq, w.T, w.topk), dtype=torch.float32, device=dev)
     out = torch.empty_like(x["q"])
     lse = torch.empty((w.B, w.Hq, w.T), dtype=torch.float32, device=dev)
-    p = H.make_params(w.B, w.T, w.L, w.Hq, w.Hkv, w.d, w.S, w.topk, w.W)
-    nws = H.workspace_size(p, H.OP_ATTN_FWD)
-    ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def step(mark):
         H.chunk_summary(x["k"], x["q_land"], w.S, k_sum=k_sum, b_sum=b_sum)
         mark()
-        H.select_topk(x["q_hat"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S, topk=w.topk, window=w.W, idx=idx)
+        H.select_topk(x["q_hat"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S, topk=w.topk, window=w.W, idx=idx,
+                      shat=shat)
         mark()
-        H.attn_fwd(x["q"], x["k"], x["v"], x["q_hat"], k_sum, b_sum, idx, S=w.S, window=w.W, out=out, lse=lse,
-                   workspace=ws if nws else None)
+        H.attn_fwd_shat(x["q"], x["k"], x["v"], idx, shat, S=w.S, window=w.W, out=out, lse=lse)
         mark()
 
     sampler = ClockSampler(physical_gpu_index(dist.local_rank))
@@ -297,7 +295,7 @@ def bench_prefill(args, dist, dev, H, peaks):
     res = {
         "workload": w, "x": x, "out": out, "lse": lse, "idx": idx, "stage_ms": [s / args.steps for s in stage_ms],
         "ms_per_step": total_ms / args.steps, "clocks": clocks, "work": work,
-        "roofline": {"bound": "tensor", "kernel": "hils_attn_fwd", "achieved": achieved,
+        "roofline": {"bound": "tensor", "kernel": "hils_attn_fwd_shat (attn_tc_kernel)", "achieved": achieved,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
                      "traffic": ATTN_TC_TRAFFIC_BYTES,
                      "note": "algorithmic flops = 4*d per (row, head, attended token); attended = window + "
@@ -474,8 +472,11 @@ def bench_prefill_local(args, dist, dev, H, peaks):
                                             window=w.W)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
+    _, _, shat = H.select_topk(x["q_hat"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S, topk=w.topk, window=w.W,
+                               with_shat=True)
+
     def step(mark):
-        H.attn_fwd(x["q"], x["k"], x["v"], x["q_hat"], k_sum, b_sum, idx, S=w.S, window=w.W, out=out, lse=lse)
+        H.attn_fwd_shat(x["q"], x["k"], x["v"], idx, shat, S=w.S, window=w.W, out=out, lse=lse)
         mark()
 
     steps = max(1, min(args.steps, 10))
@@ -485,7 +486,7 @@ def bench_prefill_local(args, dist, dev, H, peaks):
     tf = work["attn_flops"] / (ms / 1e3) / 1e12
     return {"workload": w.name, "attn_ms": ms, "achieved_tflops": tf, "frac": tf / peaks["bf16_tflops"],
             **packing_stats(w, idx),
-            "note": "hils_attn_fwd alone on its own selection; algorithmic flops as in the headline"}
+            "note": "hils_attn_fwd_shat alone on its own selection; algorithmic flops as in the headline"}
 
 
 def packing_stats(w: W.Workload, idx) -> dict:
@@ -663,6 +664,10 @@ def profile_case(args):
             mass = torch.empty((w.B, w.Hq, w.T, w.Nc), dtype=torch.float32, device=dev)
             fn = lambda: H.bsa_select_topk(x["q"], x["k"], S=w.S, topk=w.topk, window=w.W, idx=idx, mass=mass)
         elif st == "attn":
+            _, _, shat = H.select_topk(x["q_hat"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S, topk=w.topk, window=w.W,
+                                       with_shat=True)
+            fn = lambda: H.attn_fwd_shat(x["q"], x["k"], x["v"], idx, shat, S=w.S, window=w.W, out=out, lse=lse)
+        elif st == "attn_gather":
             fn = lambda: H.attn_fwd(x["q"], x["k"], x["v"], x["q_hat"], k_sum, b_sum, idx, S=w.S, window=w.W,
                                     out=out, lse=lse)
         else:
@@ -702,7 +707,8 @@ def main():
     ap.add_argument("--impl", default="hils", choices=("hils", "reference"))
     ap.add_argument("--quick", action="store_true", help="headline only (no decode sweep / training blocks)")
     ap.add_argument("--profile",
-                    choices=("summary", "select", "select_qcal", "attn", "decode", "decode_multi", "bwd", "bsa"),
+                    choices=("summary", "select", "select_qcal", "attn", "attn_gather", "decode", "decode_multi", "bwd",
+                             "bsa"),
                     help="run --steps untimed launches of one stage for an ncu capture; no bench line")
     args = ap.parse_args()
     if args.profile:
@@ -753,7 +759,7 @@ def main():
             "data": "synthetic",
             "config": base_config(w, dist.world),
             "stage_ms": {"chunk_summary": pre["stage_ms"][0], "select_topk": pre["stage_ms"][1],
-                         "attn_fwd": pre["stage_ms"][2]},
+                         "attn_fwd_shat": pre["stage_ms"][2]},
             "roofline": pre["roofline"],
             "packing": packing_stats(w, pre["idx"]),
             "cpu_baseline": cpu,

@@ -1,23 +1,23 @@
 // Stages (c)+(d) on the tensor cores: per-chunk attention and Eq. 10 fusion, prefill form, bf16, d 128,
 // chunk size 64 ("Hierarchical Sparse Attention Done Right", Sec. 3 RQ2 / Eq. 10; Sec. 4 kernel).
 //
-// Two launches:
-//  1. gather (select_tc.cu, same tcgen05 GEMM as the selection): each row's ids canonicalised (valid,
-//     distinct, ascending) and their retrieval scores s^ written to the workspace.
-//  2. this kernel. CTA = 128 rows = 128/G queries x G heads of one KV group (row = query*G + head), so
-//     the heads of a group share every K/V tile. The tiles it visits are the union of the queries'
-//     window chunks and selected chunks (the paper's query packing over the union, Fig. 4b), in
-//     descending chunk order so that window tiles come first.
-//       warp 0     TMA producer: Q once (3-D map, rows query-major), then K and V tiles (2-D maps,
-//                  128-byte swizzle) into a 3-stage ring.
-//       warp 1     MMA issuer: S = Q K^T (M 128, N 64, K 128) into one of two TMEM S buffers, then
-//                  O += P V (M 128, N 128, K 64) with V read MN-major; O lives in TMEM throughout.
-//       warps 2-5  one row each (the row's TMEM lane): per tile the row is a window row (logits
-//                  masked to its window), a selecting row (logits s_j - L_c + s^_c with L_c the
-//                  intra-chunk LSE, so the chunk carries mass exp(s^_c)), or neither (P = 0).
-//                  P is written to shared memory in the swizzled K-major layout. The running max
-//                  starts at max s^ over the row's chunks, which no chunk tile can exceed; only a
-//                  window logit more than 8 above it rescales the row of O in TMEM.
+// Launches: hils_attn_fwd first runs a gather (select_tc.cu, the selection's tcgen05 GEMM) that writes
+// each row's ids in canonical form (valid, distinct, ascending) and their retrieval scores s^ to the
+// workspace; hils_attn_fwd_shat is given both by the selection and launches this kernel alone.
+//  CTA = 128 rows = 128/G queries x G heads of one KV group (row = query*G + head), so the heads of a
+//  group share every K/V tile. The tiles it visits are the union of the queries' window chunks and
+//  selected chunks (the paper's query packing over the union, Fig. 4b), in descending chunk order so
+//  that window tiles come first.
+//    warp 0     TMA producer: Q once (3-D map, rows query-major), then K and V tiles (2-D maps, 128-byte
+//               swizzle) into two-stage K and V rings.
+//    warp 1     MMA issuer: S = Q K^T (M 128, N 64, K 128) into one of two TMEM S buffers, then
+//               O += P V (M 128, N 128, K 64) with P read from TMEM and V MN-major from shared memory;
+//               O lives in TMEM throughout.
+//    warps 2-5  one row each (the row's TMEM lane): per tile the row is a window row (logits masked to
+//               its window), a selecting row (logits s_j - L_c + s^_c with L_c the intra-chunk LSE, so
+//               the chunk carries mass exp(s^_c)), or neither (P = 0). P (bf16) overwrites its S buffer
+//               in TMEM. The running max starts at max s^ over the row's chunks, which no chunk tile can
+//               exceed; only a window logit more than 8 above it rescales the row of O in TMEM.
 //  Epilogue: O / l to bf16, lse = m + log l.
 #include "internal.h"
 #include "tcgen05.cuh"
@@ -117,13 +117,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     int ns = 0;
     float m2 = -INFINITY;  // running max, log2 units
     if (valid) {
+        // The ids must be in canonical form: candidates (c < lpos / S) strictly ascending, then -1. A row
+        // that is not keeps its canonical prefix and raises the call's error word.
+        const int n_r = lpos / S;
+        bool canon = true;
+        int prev = -1;
         for (int t = 0; t < K; ++t) {
             const int c = row_idx[t];
-            if (c < 0) break;
+            if (c == -1) {
+                for (int t2 = t + 1; t2 < K; ++t2) canon = canon && row_idx[t2] == -1;
+                break;
+            }
+            if (c <= prev || c >= n_r) {
+                canon = false;
+                break;
+            }
+            prev = c;
             ++ns;
             m2 = fmaxf(m2, row_sh[t] * kLog2e);
             atomicOr(&bitmap[c >> 5], 1u << (c & 31));
         }
+        if (!canon) atomicOr(&g_attn_tc_errors, 2u);
     }
     if (tid == 0) {
         const int ilast = min(D.T, i0 + QT) - 1;
@@ -425,14 +439,10 @@ unsigned int attn_tc_error_flags(bool clear) {
     return v;
 }
 
-cudaError_t launch_attn_fwd_tc(const Dims &D, const void *q, const void *k, const void *v, const void *q_hat,
-                               const void *k_sum, const float *b_sum, const int *idx, void *out, float *lse,
-                               void *ws, cudaStream_t stream) {
-    unsigned char *w = (unsigned char *)ws;
-    int *ws_idx = (int *)w;
-    float *ws_shat = (float *)(w + (((size_t)D.B * D.Hkv * D.T * D.topk * sizeof(int) + 255) & ~(size_t)255));
-    cudaError_t e = launch_gather_shat_tc(D, q_hat, k_sum, b_sum, idx, ws_idx, ws_shat, stream);
-    if (e != cudaSuccess) return e;
+namespace {
+
+cudaError_t launch_attn_tc(const Dims &D, const void *q, const void *k, const void *v, const int *ids,
+                           const float *shat, void *out, float *lse, cudaStream_t stream) {
     CUtensorMap qmap, kmap, vmap;
     const int QT = 128 / D.G;
     if (!make_tmap_bf16_3d(&qmap, q, 128, (uint64_t)D.B * D.Hq, (uint64_t)D.T, (uint64_t)D.T * 128 * 2, 128 * 2, D.G,
@@ -443,8 +453,36 @@ cudaError_t launch_attn_fwd_tc(const Dims &D, const void *q, const void *k, cons
     const size_t smem = 1024 + kQBytes + 2 * kStages * kTileBytes;
     cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     dim3 grid((D.T + QT - 1) / QT, D.Hkv, D.B);
-    attn_tc_kernel<<<grid, kThreads, smem, stream>>>(qmap, kmap, vmap, D, ws_idx, ws_shat, (__nv_bfloat16 *)out, lse);
+    attn_tc_kernel<<<grid, kThreads, smem, stream>>>(qmap, kmap, vmap, D, ids, shat, (__nv_bfloat16 *)out, lse);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_fwd_tc(const Dims &D, const void *q, const void *k, const void *v, const void *q_hat,
+                               const void *k_sum, const float *b_sum, const int *idx, void *out, float *lse,
+                               void *ws, cudaStream_t stream) {
+    unsigned char *w = (unsigned char *)ws;
+    int *ws_idx = (int *)w;
+    float *ws_shat = (float *)(w + (((size_t)D.B * D.Hkv * D.T * D.topk * sizeof(int) + 255) & ~(size_t)255));
+    cudaError_t e = launch_gather_shat_tc(D, q_hat, k_sum, b_sum, idx, ws_idx, ws_shat, stream);
+    if (e != cudaSuccess) return e;
+    return launch_attn_tc(D, q, k, v, ws_idx, ws_shat, out, lse, stream);
+}
+
+// Ids in canonical form with their retrieval scores given (as hils_select_topk writes them with shat):
+// no gather, and no limit of 128 candidates per row.
+bool attn_fwd_shat_supported(const Dims &D, int dtype) {
+    if (dtype != HILS_BF16 || D.d != 128 || D.S != 64 || D.topk > 32 || (128 % D.G) != 0 || D.G > 128) return false;
+    const int QT = 128 / D.G;
+    const int nchunks = (D.L + D.S - 1) / D.S;
+    const int max_list = (D.W + 2 * D.S + QT) / D.S + 2 + QT * D.topk;
+    return nchunks <= 32 * kBitmapWords && max_list <= kListCap;
+}
+
+cudaError_t launch_attn_fwd_tc_shat(const Dims &D, const void *q, const void *k, const void *v, const int *idx,
+                                    const float *shat, void *out, float *lse, cudaStream_t stream) {
+    return launch_attn_tc(D, q, k, v, idx, shat, out, lse, stream);
 }
 
 }  // namespace hils

@@ -26,13 +26,17 @@ size_t attn_fwd_tc_workspace(const Dims &D);
 hils_status check_device_errors();
 bool select_tc_supported(const Dims &D, int dtype);
 cudaError_t launch_select_tc(const Dims &D, const void *q_hat, const void *k_sum, const float *b_sum, int *idx,
-                             float *gap, cudaStream_t stream);
+                             float *gap, float *shat, cudaStream_t stream);
 unsigned int select_tc_error_flags(bool clear);
 unsigned int summary_error_flags(bool clear);
 unsigned int attn_bwd_tc_error_flags(bool clear);
 unsigned int bsa_error_flags(bool clear);
 cudaError_t launch_select_tc_qcal(const Dims &D, const void *q, const void *w_down, const void *w_up,
-                                  const void *k_sum, const float *b_sum, int *idx, float *gap, cudaStream_t stream);
+                                  const void *k_sum, const float *b_sum, int *idx, float *gap, float *shat,
+                                  cudaStream_t stream);
+bool attn_fwd_shat_supported(const Dims &D, int dtype);
+cudaError_t launch_attn_fwd_tc_shat(const Dims &D, const void *q, const void *k, const void *v, const int *idx,
+                                    const float *shat, void *out, float *lse, cudaStream_t stream);
 int bsa_max_candidates(const Dims &D);
 cudaError_t launch_bsa_select_topk(const Dims &D, int dtype, const void *q, const void *k, int *idx, float *gap,
                                    float *mass, cudaStream_t stream);
@@ -113,9 +117,13 @@ hils_status check_device_errors() {
     if (select_tc_error_flags(true) != 0)
         return fail(HILS_ERR_TIMEOUT, "hils_check: a tensor-core selection tile's wait expired; that call's ids are "
                     "invalid");
-    if (attn_tc_error_flags(true) != 0)
+    const unsigned int af = attn_tc_error_flags(true);
+    if (af & 1u)
         return fail(HILS_ERR_TIMEOUT, "hils_check: a tensor-core attention tile's wait expired; that call's output "
                     "is invalid");
+    if (af & 2u)
+        return fail(HILS_ERR_INVALID_ARG, "hils_check: hils_attn_fwd_shat was given a row of ids not in canonical "
+                    "form (candidate ids strictly ascending, then -1); that call's output is invalid");
     if (attn_bwd_tc_error_flags(true) != 0)
         return fail(HILS_ERR_TIMEOUT, "hils_check: a tensor-core backward tile's wait expired; that call's "
                     "gradients are invalid");
@@ -205,7 +213,8 @@ hils_status hils_chunk_summary_shared_query(const hils_params *p, const void *k,
 }
 
 hils_status hils_select_topk(const hils_params *p, const void *q_hat, const void *k_sum, const float *b_sum,
-                             int32_t *idx, float *gap, void *workspace, size_t workspace_bytes, hils_stream_t stream) {
+                             int32_t *idx, float *gap, float *shat, void *workspace, size_t workspace_bytes,
+                             hils_stream_t stream) {
     const char *fn = "hils_select_topk";
     Dims D;
     hils_status st = resolve(p, fn, &D);
@@ -217,19 +226,20 @@ hils_status hils_select_topk(const hils_params *p, const void *q_hat, const void
         HILS_REQUIRE_PTR(b_sum);
     }
     if (gap != nullptr && !aligned16(gap)) return fail(HILS_ERR_INVALID_ARG, "%s: gap is not 16-byte aligned", fn);
+    if (shat != nullptr && !aligned16(shat)) return fail(HILS_ERR_INVALID_ARG, "%s: shat is not 16-byte aligned", fn);
     if (select_smem_bytes(D) > kMaxSmem)
         return fail(HILS_ERR_UNSUPPORTED, "%s: %d chunks x %d heads exceed one CTA's shared memory; use hils_decode",
                     fn, D.Nc, D.G);
     st = check_ws(fn, workspace, workspace_bytes, 0);
     if (st != HILS_OK) return st;
     if (select_tc_supported(D, p->dtype))
-        return cuda_status(launch_select_tc(D, q_hat, k_sum, b_sum, idx, gap, (cudaStream_t)stream), fn);
-    return cuda_status(launch_select_topk(D, p->dtype, q_hat, k_sum, b_sum, idx, gap, (cudaStream_t)stream), fn);
+        return cuda_status(launch_select_tc(D, q_hat, k_sum, b_sum, idx, gap, shat, (cudaStream_t)stream), fn);
+    return cuda_status(launch_select_topk(D, p->dtype, q_hat, k_sum, b_sum, idx, gap, shat, (cudaStream_t)stream), fn);
 }
 
 hils_status hils_select_topk_qcal(const hils_params *p, const void *q, const void *w_down, const void *w_up,
                                   int32_t rank, const void *k_sum, const float *b_sum, int32_t *idx, float *gap,
-                                  hils_stream_t stream) {
+                                  float *shat, hils_stream_t stream) {
     const char *fn = "hils_select_topk_qcal";
     Dims D;
     hils_status st = resolve(p, fn, &D);
@@ -245,7 +255,9 @@ hils_status hils_select_topk_qcal(const hils_params *p, const void *q, const voi
     HILS_REQUIRE_PTR(b_sum);
     HILS_REQUIRE_PTR(idx);
     if (gap != nullptr && !aligned16(gap)) return fail(HILS_ERR_INVALID_ARG, "%s: gap is not 16-byte aligned", fn);
-    return cuda_status(launch_select_tc_qcal(D, q, w_down, w_up, k_sum, b_sum, idx, gap, (cudaStream_t)stream), fn);
+    if (shat != nullptr && !aligned16(shat)) return fail(HILS_ERR_INVALID_ARG, "%s: shat is not 16-byte aligned", fn);
+    return cuda_status(launch_select_tc_qcal(D, q, w_down, w_up, k_sum, b_sum, idx, gap, shat, (cudaStream_t)stream),
+                       fn);
 }
 
 hils_status hils_bsa_select_topk(const hils_params *p, const void *q, const void *k, int32_t *idx, float *gap,
@@ -291,6 +303,25 @@ hils_status hils_attn_fwd(const hils_params *p, const void *q, const void *k, co
             launch_attn_fwd_tc(D, q, k, v, q_hat, k_sum, b_sum, idx, out, lse, workspace, (cudaStream_t)stream), fn);
     return cuda_status(
         launch_attn_fwd_simt(D, p->dtype, q, k, v, q_hat, k_sum, b_sum, idx, out, lse, (cudaStream_t)stream), fn);
+}
+
+hils_status hils_attn_fwd_shat(const hils_params *p, const void *q, const void *k, const void *v, const int32_t *idx,
+                               const float *shat, void *out, float *lse, hils_stream_t stream) {
+    const char *fn = "hils_attn_fwd_shat";
+    Dims D;
+    hils_status st = resolve(p, fn, &D);
+    if (st != HILS_OK) return st;
+    if (!attn_fwd_shat_supported(D, p->dtype))
+        return fail(HILS_ERR_UNSUPPORTED, "%s: needs bf16, d 128, S 64, 128 %% G == 0, topk <= 32 and at most 8192 "
+                    "chunks (otherwise call hils_attn_fwd)", fn);
+    HILS_REQUIRE_PTR(q);
+    HILS_REQUIRE_PTR(k);
+    HILS_REQUIRE_PTR(v);
+    HILS_REQUIRE_PTR(idx);
+    HILS_REQUIRE_PTR(shat);
+    HILS_REQUIRE_PTR(out);
+    HILS_REQUIRE_PTR(lse);
+    return cuda_status(launch_attn_fwd_tc_shat(D, q, k, v, idx, shat, out, lse, (cudaStream_t)stream), fn);
 }
 
 hils_status hils_decode(const hils_params *p, const void *q, const void *q_hat, const void *k_cache,

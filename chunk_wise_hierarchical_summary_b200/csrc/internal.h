@@ -14,7 +14,7 @@ cudaError_t launch_chunk_summary(const Dims &D, int dtype, const void *k, const 
 
 size_t select_smem_bytes(const Dims &D);
 cudaError_t launch_select_topk(const Dims &D, int dtype, const void *q_hat, const void *k_sum, const float *b_sum,
-                               int *idx, float *gap, cudaStream_t stream);
+                               int *idx, float *gap, float *shat, cudaStream_t stream);
 
 cudaError_t launch_attn_fwd(const Dims &D, int dtype, const void *q, const void *k, const void *v, const void *q_hat,
                             const void *k_sum, const float *b_sum, const int *idx, void *out, float *lse,

@@ -5,7 +5,8 @@
 //   s^_{h,c} = tau * q^_{h,i} . k'_{h,c} + b'_{h,c}          (each head h of the group; fp32)
 //   g_c = max_h (s^_{h,c} - LSE_{c'<n} s^_{h,c'})            (per-head normalised weight, max over heads)
 // then a block-wide bitonic sort of the keys (g desc, c asc) gives the top-min(k, n) and the gap
-// g_(k) - g_(k+1). The summary rows are read with half-warp-per-row 16-byte loads.
+// g_(k) - g_(k+1); optionally each head's s^ of the kept ids. The summary rows are read with
+// half-warp-per-row 16-byte loads.
 #include "internal.h"
 
 namespace hils {
@@ -16,7 +17,7 @@ constexpr int kSelectThreads = 256;
 template <typename T>
 __global__ void __launch_bounds__(kSelectThreads)
 select_kernel(Dims D, const T *__restrict__ q_hat, const T *__restrict__ k_sum, const float *__restrict__ b_sum,
-              int *__restrict__ idx, float *__restrict__ gap) {
+              int *__restrict__ idx, float *__restrict__ gap, float *__restrict__ shat) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int i = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int d = D.d, G = D.G, K = D.topk;
@@ -24,8 +25,14 @@ select_kernel(Dims D, const T *__restrict__ q_hat, const T *__restrict__ k_sum, 
     const int n = window_left(pos, D.W, D.S) / D.S;
     int *row = idx + (((size_t)b * D.Hkv + g) * D.T + i) * K;
     float *gp = gap ? gap + ((size_t)b * D.Hkv + g) * D.T + i : nullptr;
+    // shat (nullable): each head's s^ of the kept ids, in the order of row; -inf in the unused slots
+    auto shat_row = [&](int hh) { return shat + (((size_t)b * D.Hq + g * G + hh) * D.T + i) * K; };
     if (n == 0) {
-        for (int t = threadIdx.x; t < K; t += blockDim.x) row[t] = -1;
+        for (int t = threadIdx.x; t < K; t += blockDim.x) {
+            row[t] = -1;
+            if (shat)
+                for (int hh = 0; hh < G; ++hh) shat_row(hh)[t] = -INFINITY;
+        }
         if (gp && threadIdx.x == 0) *gp = INFINITY;
         return;
     }
@@ -100,8 +107,12 @@ select_kernel(Dims D, const T *__restrict__ q_hat, const T *__restrict__ k_sum, 
             int rank = 0;
             for (int u = 0; u < kk; ++u) rank += desc_key_index(keys[u]) < me;
             row[rank] = (int)me;
+            if (shat)
+                for (int hh = 0; hh < G; ++hh) shat_row(hh)[rank] = sc[hh * n + me];
         } else {
             row[t] = -1;
+            if (shat)
+                for (int hh = 0; hh < G; ++hh) shat_row(hh)[t] = -INFINITY;
         }
     }
 }
@@ -115,18 +126,19 @@ size_t select_smem_bytes(const Dims &D) {
 }
 
 cudaError_t launch_select_topk(const Dims &D, int dtype, const void *q_hat, const void *k_sum, const float *b_sum,
-                               int *idx, float *gap, cudaStream_t stream) {
+                               int *idx, float *gap, float *shat, cudaStream_t stream) {
     const size_t smem = select_smem_bytes(D);
     dim3 grid(D.T, D.Hkv, D.B);
     if (dtype == HILS_BF16) {
         auto kern = select_kernel<__nv_bfloat16>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         kern<<<grid, kSelectThreads, smem, stream>>>(D, (const __nv_bfloat16 *)q_hat, (const __nv_bfloat16 *)k_sum,
-                                                     b_sum, idx, gap);
+                                                     b_sum, idx, gap, shat);
     } else {
         auto kern = select_kernel<float>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        kern<<<grid, kSelectThreads, smem, stream>>>(D, (const float *)q_hat, (const float *)k_sum, b_sum, idx, gap);
+        kern<<<grid, kSelectThreads, smem, stream>>>(D, (const float *)q_hat, (const float *)k_sum, b_sum, idx, gap,
+                                                     shat);
     }
     return cudaGetLastError();
 }

@@ -34,6 +34,39 @@ constexpr int kWdRow = 272;         // W_down row (128 bf16) padded: conflict-fr
 constexpr int kWuRow = 80;          // W_up row (32 bf16) padded
 constexpr int kWdBytes = kRank * kWdRow;
 constexpr int kWuBytes = 128 * kWuRow;
+constexpr int kScoreRow = 129;      // floats per row of exact group scores (odd: conflict-free columns)
+template <int K1MAX>
+constexpr int kListBytes = (kRows * (4 * K1MAX + 1) * 4 + 15) & ~15;
+// Shared memory of the selection: the two operand stages, reused after the MMAs for the per-thread
+// sorted key lists and the exact group scores.
+template <int K1MAX>
+constexpr size_t select_dyn_smem() {
+    const size_t lists = (size_t)kListBytes<K1MAX> + (size_t)kRows * kScoreRow * 4;
+    return 1024 + (lists > 2 * (size_t)kStageBytes ? lists : 2 * (size_t)kStageBytes);
+}
+
+// 32-bit selection key whose ascending order is (score descending, chunk ascending) for chunks < 128:
+// the high 25 bits are the order-preserving image of the score cut to 16 mantissa bits, the low 7 the
+// chunk. Two scores |v| < 64 apart by more than 2^-10 keep their order; closer ones order by chunk.
+__device__ __forceinline__ uint32_t sel_key32(float v, uint32_t c) { return (~float_order_key(v) & ~127u) | c; }
+
+// Ascending bitonic sort of 32 keys held by one thread (compile-time indices: registers only).
+__device__ __forceinline__ void sort32_u32(uint32_t (&k)[32]) {
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1)
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int jx = i ^ stride;
+                if (jx > i) {
+                    const uint32_t a = k[i], b = k[jx];
+                    const bool up = (i & size) == 0;
+                    k[i] = up ? min(a, b) : max(a, b);
+                    k[jx] = up ? max(a, b) : min(a, b);
+                }
+            }
+}
 
 // q -> q^ = q + W_up (W_down q) for rows rb .. rb+15 of a 128 x 128 bf16 tile in the 128-byte-swizzled
 // K-major layout (two 64-column halves of 16 KiB), in place. One warp.
@@ -100,14 +133,15 @@ template <int K1MAX, int GATHER, int QCAL>
 __global__ void __launch_bounds__(kThreads, 1)
 select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, Dims D,
                  const float *__restrict__ b_sum, int *__restrict__ idx, float *__restrict__ gap,
-                 int *__restrict__ ws_idx, float *__restrict__ ws_shat, const __nv_bfloat16 *__restrict__ w_down,
-                 const __nv_bfloat16 *__restrict__ w_up) {
+                 float *__restrict__ shat, int *__restrict__ ws_idx, float *__restrict__ ws_shat,
+                 const __nv_bfloat16 *__restrict__ w_down, const __nv_bfloat16 *__restrict__ w_up) {
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t tma_bar[2], mma_bar[2], done_bar, qcal_bar[2];
     __shared__ __align__(16) unsigned char wsm[QCAL ? kWdBytes + kWuBytes : 16];
     __shared__ uint32_t s_tmem;
     __shared__ float bs[4][kRows];
     __shared__ float lse[4][kRows];
+    __shared__ uint32_t smask[kRows][4];  // selected set of each row (128-bit mask)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int i0 = blockIdx.x * kRows, g = blockIdx.y, b = blockIdx.z;
     const int G = D.G, K = D.topk;
@@ -313,94 +347,125 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
     __syncthreads();
     tc_fence_after();
 
-    // Phase 2: group scores of column block j, best K1MAX per row kept sorted in registers.
-    uint64_t top[K1MAX];
+    // Phase 2: group scores of column block j (32 candidates a thread) as 32-bit keys, sorted in
+    // registers; the exact scores go to shared memory for the gap. The operand stages are dead once every
+    // MMA has completed: [0, list bytes) holds the lists, the score rows follow.
+    constexpr int kRowKeys = 4 * K1MAX + 1;  // odd: neighbouring rows' lists fall in different banks
+    uint32_t *lists = reinterpret_cast<uint32_t *>(base);
+    float *gsc = reinterpret_cast<float *>(base + kListBytes<K1MAX>);  // [kRows][kScoreRow]
+    {
+        uint32_t key[32];
 #pragma unroll
-    for (int t = 0; t < K1MAX; ++t) top[t] = ~0ull;
-#pragma unroll 1
-    for (int half = 0; half < 2; ++half) {
-        const int cb = 32 * j + 16 * half;  // first column of this 16-wide piece
-        float gv[16];
+        for (int half = 0; half < 2; ++half) {
+            const int cb = 32 * j + 16 * half;  // first column of this 16-wide piece
+            float gv[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) gv[e] = -INFINITY;
-        for (int hh = 0; hh < G; ++hh) {
-            float v[16];
-            tmem_ld16(lane_base + hh * 128 + cb, v);
-            tmem_wait_ld();
-            const float l = lse[hh][r];
+            for (int e = 0; e < 16; ++e) gv[e] = -INFINITY;
+            for (int hh = 0; hh < G; ++hh) {
+                float v[16];
+                tmem_ld16(lane_base + hh * 128 + cb, v);
+                tmem_wait_ld();
+                const float l = lse[hh][r];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) gv[e] = fmaxf(gv[e], fmaf(D.tau, v[e], bs[hh][cb + e]) - l);
-        }
+                for (int e = 0; e < 16; ++e) gv[e] = fmaxf(gv[e], fmaf(D.tau, v[e], bs[hh][cb + e]) - l);
+            }
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const int c = cb + e;
-            if (c < n_r) {
-                uint64_t x = desc_value_key(gv[e], (uint32_t)c);
-                if (x < top[K1MAX - 1]) {
-#pragma unroll
-                    for (int t = 0; t < K1MAX; ++t) {
-                        if (x < top[t]) {
-                            const uint64_t y = top[t];
-                            top[t] = x;
-                            x = y;
-                        }
-                    }
-                }
+            for (int e = 0; e < 16; ++e) {
+                const int c = cb + e;
+                key[16 * half + e] = (c < n_r) ? sel_key32(gv[e], (uint32_t)c) : 0xffffffffu;
+                gsc[r * kScoreRow + c] = gv[e];
             }
         }
+        sort32_u32(key);
+#pragma unroll
+        for (int t = 0; t < K1MAX; ++t) lists[r * kRowKeys + j * K1MAX + t] = t < 32 ? key[t] : 0xffffffffu;
     }
     tc_fence_before();
-    __syncthreads();  // every TMEM read done; operand tiles are dead: reuse them for the lists
-    // [128 rows][4 blocks][K1MAX], rows padded by one key so that neighbouring rows' lists fall in
-    // different shared-memory banks
-    constexpr int kRowKeys = 4 * K1MAX + 1;
-    uint64_t *lists = reinterpret_cast<uint64_t *>(base);
-#pragma unroll
-    for (int t = 0; t < K1MAX; ++t) lists[(size_t)r * kRowKeys + j * K1MAX + t] = top[t];
     __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, ncols);
-    }
 
-    // Phase 3: merge the four sorted lists of a row.
+    // Phase 3: one thread per row merges its four sorted lists: the first min(K + 1, n) keys give the
+    // selected set (a 128-bit mask, read out ascending) and the k-th and (k+1)-th ids for the gap.
     if (tid < kRows) {
         const int rr = tid, ii = i0 + rr;
+        uint32_t m0 = 0u, m1 = 0u, m2 = 0u, m3 = 0u;
         if (ii < D.T) {
             const int nn = window_left(D.q_pos0 + ii, D.W, D.S) / D.S;
-            const uint64_t *L = lists + (size_t)rr * kRowKeys;
+            const uint32_t *Lr = lists + rr * kRowKeys;
             int p0 = 0, p1 = 0, p2 = 0, p3 = 0;
             const int need = min(K + 1, nn);
-            uint32_t ids[K1MAX];
-            float vk = 0.f, vk1 = 0.f;
+            int ck = 0, ck1 = 0;
             for (int t = 0; t < need; ++t) {
-                const uint64_t a0 = p0 < K1MAX ? L[p0] : ~0ull, a1 = p1 < K1MAX ? L[K1MAX + p1] : ~0ull;
-                const uint64_t a2 = p2 < K1MAX ? L[2 * K1MAX + p2] : ~0ull, a3 = p3 < K1MAX ? L[3 * K1MAX + p3] : ~0ull;
-                uint64_t m01 = a0 < a1 ? a0 : a1, m23 = a2 < a3 ? a2 : a3;
-                const uint64_t mm = m01 < m23 ? m01 : m23;
+                const uint32_t a0 = p0 < K1MAX ? Lr[p0] : 0xffffffffu, a1 = p1 < K1MAX ? Lr[K1MAX + p1] : 0xffffffffu;
+                const uint32_t a2 = p2 < K1MAX ? Lr[2 * K1MAX + p2] : 0xffffffffu;
+                const uint32_t a3 = p3 < K1MAX ? Lr[3 * K1MAX + p3] : 0xffffffffu;
+                const uint32_t mm = min(min(a0, a1), min(a2, a3));
                 if (mm == a0) ++p0;
                 else if (mm == a1) ++p1;
                 else if (mm == a2) ++p2;
                 else ++p3;
-                if (t < K) ids[t] = desc_key_index(mm);
-                if (t == K - 1) vk = desc_key_value(mm);
-                if (t == K) vk1 = desc_key_value(mm);
-            }
-            const int kk = min(K, nn);
-            // ids ascending (insertion sort of at most K1MAX - 1 values)
-            for (int a = 1; a < kk; ++a) {
-                const uint32_t x = ids[a];
-                int c = a - 1;
-                while (c >= 0 && ids[c] > x) {
-                    ids[c + 1] = ids[c];
-                    --c;
+                const int c = (int)(mm & 127u);
+                if (t < K) {
+                    const uint32_t bit = 1u << (c & 31);
+                    const int w = c >> 5;
+                    m0 |= (w == 0) ? bit : 0u;
+                    m1 |= (w == 1) ? bit : 0u;
+                    m2 |= (w == 2) ? bit : 0u;
+                    m3 |= (w == 3) ? bit : 0u;
                 }
-                ids[c + 1] = x;
+                if (t == K - 1) ck = c;
+                if (t == K) ck1 = c;
             }
             int *row = idx + (((size_t)b * D.Hkv + g) * D.T + ii) * K;
-            for (int t = 0; t < K; ++t) row[t] = t < kk ? (int)ids[t] : -1;
-            if (gap) gap[((size_t)b * D.Hkv + g) * D.T + ii] = (nn > K) ? vk - vk1 : INFINITY;
+            int ns = 0;
+            const uint32_t words[4] = {m0, m1, m2, m3};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                uint32_t x = words[w];
+                while (x) {
+                    row[ns++] = 32 * w + __ffs(x) - 1;
+                    x &= x - 1u;
+                }
+            }
+            for (int t = ns; t < K; ++t) row[t] = -1;
+            if (gap)
+                gap[((size_t)b * D.Hkv + g) * D.T + ii] =
+                    (nn > K) ? gsc[rr * kScoreRow + ck] - gsc[rr * kScoreRow + ck1] : INFINITY;
         }
+        smask[rr][0] = m0;
+        smask[rr][1] = m1;
+        smask[rr][2] = m2;
+        smask[rr][3] = m3;
+    }
+
+    // Phase 4 (optional): each head's retrieval score s^ = tau D + b' of the selected ids, in id order,
+    // -inf in the unused slots.
+    if (shat != nullptr) {
+        __syncthreads();
+        if (j < G) {  // warp-uniform: every lane executes the TMEM loads
+            const int hh = j;
+            float *dst = shat + (((size_t)b * D.Hq + g * G + hh) * D.T + (i < D.T ? i : 0)) * K;
+            int u = 0;
+#pragma unroll 1
+            for (int t = 0; t < 4; ++t) {
+                float v[32];
+                tmem_ld32(lane_base + hh * 128 + 32 * t, v);
+                tmem_wait_ld();
+                const uint32_t m = smask[r][t];
+                if (i < D.T) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if ((m >> e) & 1u) dst[u++] = fmaf(D.tau, v[e], bs[hh][32 * t + e]);
+                }
+            }
+            if (i < D.T)
+                for (int t = u; t < K; ++t) dst[t] = -INFINITY;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, ncols);
     }
     if (!ok && tid == 0) atomicOr(&g_select_tc_errors, 2u);
 }
@@ -423,49 +488,49 @@ unsigned int select_tc_error_flags(bool clear) {
     return v;
 }
 
+namespace {
+
+template <int K1MAX, int QCAL>
+void launch_select_variant(const CUtensorMap &qmap, const CUtensorMap &kmap, const Dims &D, const float *b_sum,
+                           int *idx, float *gap, float *shat, const __nv_bfloat16 *wd, const __nv_bfloat16 *wu,
+                           cudaStream_t stream) {
+    const size_t smem = select_dyn_smem<K1MAX>();
+    dim3 grid((D.T + kRows - 1) / kRows, D.Hkv, D.B);
+    cudaFuncSetAttribute(select_tc_kernel<K1MAX, 0, QCAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    select_tc_kernel<K1MAX, 0, QCAL><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap, shat, nullptr,
+                                                                        nullptr, wd, wu);
+}
+
+}  // namespace
+
 cudaError_t launch_select_tc(const Dims &D, const void *q_hat, const void *k_sum, const float *b_sum, int *idx,
-                             float *gap, cudaStream_t stream) {
+                             float *gap, float *shat, cudaStream_t stream) {
     CUtensorMap qmap, kmap;
     if (!make_tmap_bf16_2d(&qmap, q_hat, (uint64_t)D.B * D.Hq * D.T, 128, 128, 128) ||
         !make_tmap_bf16_2d(&kmap, k_sum, (uint64_t)D.B * D.Hq * D.Nc, 128, 128, 128))
         return cudaErrorInvalidValue;
-    dim3 grid((D.T + kRows - 1) / kRows, D.Hkv, D.B);
-    if (D.topk <= 16) {
-        const size_t smem = 1024 + 2 * (size_t)kStageBytes;  // lists: 128 * 69 * 8 = 69 KiB fit in the stages
-        cudaFuncSetAttribute(select_tc_kernel<17, 0, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        select_tc_kernel<17, 0, 0><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap, nullptr, nullptr,
-                                                                     nullptr, nullptr);
-    } else {
-        const size_t smem = 1024 + (size_t)kRows * (4 * 33 + 1) * 8;  // 133 KiB of lists > the two stages
-        cudaFuncSetAttribute(select_tc_kernel<33, 0, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        select_tc_kernel<33, 0, 0><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap, nullptr, nullptr,
-                                                                     nullptr, nullptr);
-    }
+    if (D.topk <= 16)
+        launch_select_variant<17, 0>(qmap, kmap, D, b_sum, idx, gap, shat, nullptr, nullptr, stream);
+    else
+        launch_select_variant<33, 0>(qmap, kmap, D, b_sum, idx, gap, shat, nullptr, nullptr, stream);
     return cudaGetLastError();
 }
 
 // The same selection from q with the Q-Cal projection fused in (rank 32, one W_down [32, 128] and
 // W_up [128, 32] pair for every head, bf16, 16-byte aligned).
 cudaError_t launch_select_tc_qcal(const Dims &D, const void *q, const void *w_down, const void *w_up,
-                                  const void *k_sum, const float *b_sum, int *idx, float *gap, cudaStream_t stream) {
+                                  const void *k_sum, const float *b_sum, int *idx, float *gap, float *shat,
+                                  cudaStream_t stream) {
     CUtensorMap qmap, kmap;
     if (!make_tmap_bf16_2d(&qmap, q, (uint64_t)D.B * D.Hq * D.T, 128, 128, 128) ||
         !make_tmap_bf16_2d(&kmap, k_sum, (uint64_t)D.B * D.Hq * D.Nc, 128, 128, 128))
         return cudaErrorInvalidValue;
-    dim3 grid((D.T + kRows - 1) / kRows, D.Hkv, D.B);
     const auto *wd = (const __nv_bfloat16 *)w_down;
     const auto *wu = (const __nv_bfloat16 *)w_up;
-    if (D.topk <= 16) {
-        const size_t smem = 1024 + 2 * (size_t)kStageBytes;
-        cudaFuncSetAttribute(select_tc_kernel<17, 0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        select_tc_kernel<17, 0, 1><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap, nullptr, nullptr,
-                                                                     wd, wu);
-    } else {
-        const size_t smem = 1024 + (size_t)kRows * (4 * 33 + 1) * 8;
-        cudaFuncSetAttribute(select_tc_kernel<33, 0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        select_tc_kernel<33, 0, 1><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, idx, gap, nullptr, nullptr,
-                                                                     wd, wu);
-    }
+    if (D.topk <= 16)
+        launch_select_variant<17, 1>(qmap, kmap, D, b_sum, idx, gap, shat, wd, wu, stream);
+    else
+        launch_select_variant<33, 1>(qmap, kmap, D, b_sum, idx, gap, shat, wd, wu, stream);
     return cudaGetLastError();
 }
 
@@ -481,7 +546,7 @@ cudaError_t launch_gather_shat_tc(const Dims &D, const void *q_hat, const void *
     const size_t smem = 1024 + 2 * (size_t)kStageBytes;
     cudaFuncSetAttribute(select_tc_kernel<17, 1, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     select_tc_kernel<17, 1, 0><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, const_cast<int *>(idx), nullptr,
-                                                                  ws_idx, ws_shat, nullptr, nullptr);
+                                                                  nullptr, ws_idx, ws_shat, nullptr, nullptr);
     return cudaGetLastError();
 }
 

@@ -28,7 +28,7 @@ OP_SUMMARY, OP_SELECT, OP_ATTN_FWD, OP_DECODE, OP_ATTN_BWD = 0, 1, 2, 3, 4
 # Every symbol include/hils.h declares (checked by the tests against the header and the library).
 EXPORTED = ("hils_workspace_size", "hils_chunk_summary", "hils_chunk_summary_shared_query", "hils_select_topk",
             "hils_select_topk_qcal", "hils_bsa_select_topk", "hils_attn_fwd", "hils_decode", "hils_attn_bwd", "hils_check", "hils_status_string", "hils_last_error",
-            "hils_version", "hils_decode_noalloc", "hils_test_wait_expiry")
+            "hils_version", "hils_decode_noalloc", "hils_test_wait_expiry", "hils_attn_fwd_shat")
 
 
 class HilsError(RuntimeError):
@@ -54,13 +54,15 @@ def _load() -> ctypes.CDLL:
     lib.hils_chunk_summary.restype = st
     lib.hils_chunk_summary_shared_query.argtypes = [P, vp, vp, ctypes.c_int32, ctypes.c_int32, vp, vp, vp]
     lib.hils_chunk_summary_shared_query.restype = st
-    lib.hils_select_topk.argtypes = [P, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.hils_select_topk.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.hils_select_topk.restype = st
     lib.hils_bsa_select_topk.argtypes = [P, vp, vp, vp, vp, vp, vp]
     lib.hils_bsa_select_topk.restype = st
-    lib.hils_select_topk_qcal.argtypes = [P, vp, vp, vp, ctypes.c_int32, vp, vp, vp, vp, vp]
+    lib.hils_select_topk_qcal.argtypes = [P, vp, vp, vp, ctypes.c_int32, vp, vp, vp, vp, vp, vp]
     lib.hils_select_topk_qcal.restype = st
     lib.hils_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.hils_attn_fwd_shat.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.hils_attn_fwd_shat.restype = st
     lib.hils_attn_fwd.restype = st
     lib.hils_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.hils_decode.restype = st
@@ -177,15 +179,7 @@ def chunk_summary_shared_query(k, q_shared, S: int, *, c_begin: int = 0, c_end: 
     return k_sum, b_sum
 
 
-def select_topk(q_hat, k_sum, b_sum, *, Hkv: int, L: int, S: int, topk: int, window: int, q_pos0: int = 0,
-                    scale: float = 0.0, with_gap: bool = False, idx=None, gap=None):
-    """GQA-shared top-k (Eq. 7, Sec. 3 RQ1, Sec. 4). q_hat [B,Hq,T,d], k_sum [B,Hq,Nc,d], b_sum [B,Hq,Nc]
-    -> idx [B,Hkv,T,topk] int32 (ascending ids, -1 padded) and, with with_gap, gap [B,Hkv,T] fp32."""
-    B, Hq, T, d = q_hat.shape
-    dev, dt = q_hat.device, q_hat.dtype
-    Nc = L // S
-    _check("k_sum", k_sum, dt, (B, Hq, Nc, d), dev)
-    _check("b_sum", b_sum, torch.float32, (B, Hq, Nc), dev)
+def _selection_outputs(B, Hq, Hkv, T, topk, dev, with_gap, with_shat, idx, gap, shat):
     if idx is None:
         idx = torch.empty((B, Hkv, T, topk), dtype=torch.int32, device=dev)
     _check("idx", idx, torch.int32, (B, Hkv, T, topk), dev)
@@ -193,17 +187,43 @@ def select_topk(q_hat, k_sum, b_sum, *, Hkv: int, L: int, S: int, topk: int, win
         gap = torch.empty((B, Hkv, T), dtype=torch.float32, device=dev)
     if gap is not None:
         _check("gap", gap, torch.float32, (B, Hkv, T), dev)
-    p = make_params(B, T, L, Hq, Hkv, d, S, topk, window, q_pos0, scale, dt)
-    ws, nws = _workspace(p, OP_SELECT, dev, None)
-    _raise(lib.hils_select_topk(ctypes.byref(p), _ptr(q_hat), _ptr(k_sum), _ptr(b_sum), _ptr(idx), _ptr(gap),
-                                _ptr(ws), nws, _stream(dev)))
+    if with_shat and shat is None:
+        shat = torch.empty((B, Hq, T, topk), dtype=torch.float32, device=dev)
+    if shat is not None:
+        _check("shat", shat, torch.float32, (B, Hq, T, topk), dev)
+    return idx, gap, shat
+
+
+def _selection_result(idx, gap, shat, with_shat):
+    if with_shat or shat is not None:
+        return idx, gap, shat
     return (idx, gap) if gap is not None else idx
 
 
+def select_topk(q_hat, k_sum, b_sum, *, Hkv: int, L: int, S: int, topk: int, window: int, q_pos0: int = 0,
+                    scale: float = 0.0, with_gap: bool = False, with_shat: bool = False, idx=None, gap=None,
+                    shat=None):
+    """GQA-shared top-k (Eq. 7, Sec. 3 RQ1, Sec. 4). q_hat [B,Hq,T,d], k_sum [B,Hq,Nc,d], b_sum [B,Hq,Nc]
+    -> idx [B,Hkv,T,topk] int32 (ascending ids, -1 padded); with with_gap also gap [B,Hkv,T] fp32 and with
+    with_shat (idx, gap or None, shat [B,Hq,T,topk] fp32: each head's s^ of the selected ids)."""
+    B, Hq, T, d = q_hat.shape
+    dev, dt = q_hat.device, q_hat.dtype
+    Nc = L // S
+    _check("k_sum", k_sum, dt, (B, Hq, Nc, d), dev)
+    _check("b_sum", b_sum, torch.float32, (B, Hq, Nc), dev)
+    idx, gap, shat = _selection_outputs(B, Hq, Hkv, T, topk, dev, with_gap, with_shat, idx, gap, shat)
+    p = make_params(B, T, L, Hq, Hkv, d, S, topk, window, q_pos0, scale, dt)
+    ws, nws = _workspace(p, OP_SELECT, dev, None)
+    _raise(lib.hils_select_topk(ctypes.byref(p), _ptr(q_hat), _ptr(k_sum), _ptr(b_sum), _ptr(idx), _ptr(gap),
+                                _ptr(shat), _ptr(ws), nws, _stream(dev)))
+    return _selection_result(idx, gap, shat, with_shat)
+
+
 def select_topk_qcal(q, w_down, w_up, k_sum, b_sum, *, Hkv: int, L: int, S: int, topk: int, window: int,
-                     q_pos0: int = 0, scale: float = 0.0, with_gap: bool = False, idx=None, gap=None):
+                     q_pos0: int = 0, scale: float = 0.0, with_gap: bool = False, with_shat: bool = False, idx=None,
+                     gap=None, shat=None):
     """select_topk with Q-Cal fused (Sec. 4): q [B,Hq,T,d], w_down [r,d], w_up [d,r] (r = 32) ->
-    idx [B,Hkv,T,topk] int32 (and gap), selected on q^ = q + W_up (W_down q)."""
+    idx [B,Hkv,T,topk] int32 (and gap, shat as select_topk), selected on q^ = q + W_up (W_down q)."""
     B, Hq, T, d = q.shape
     dev, dt = q.device, q.dtype
     r = w_down.shape[0]
@@ -212,17 +232,11 @@ def select_topk_qcal(q, w_down, w_up, k_sum, b_sum, *, Hkv: int, L: int, S: int,
     Nc = L // S
     _check("k_sum", k_sum, dt, (B, Hq, Nc, d), dev)
     _check("b_sum", b_sum, torch.float32, (B, Hq, Nc), dev)
-    if idx is None:
-        idx = torch.empty((B, Hkv, T, topk), dtype=torch.int32, device=dev)
-    _check("idx", idx, torch.int32, (B, Hkv, T, topk), dev)
-    if with_gap and gap is None:
-        gap = torch.empty((B, Hkv, T), dtype=torch.float32, device=dev)
-    if gap is not None:
-        _check("gap", gap, torch.float32, (B, Hkv, T), dev)
+    idx, gap, shat = _selection_outputs(B, Hq, Hkv, T, topk, dev, with_gap, with_shat, idx, gap, shat)
     p = make_params(B, T, L, Hq, Hkv, d, S, topk, window, q_pos0, scale, dt)
     _raise(lib.hils_select_topk_qcal(ctypes.byref(p), _ptr(q), _ptr(w_down), _ptr(w_up), r, _ptr(k_sum), _ptr(b_sum),
-                                     _ptr(idx), _ptr(gap), _stream(dev)))
-    return (idx, gap) if gap is not None else idx
+                                     _ptr(idx), _ptr(gap), _ptr(shat), _stream(dev)))
+    return _selection_result(idx, gap, shat, with_shat)
 
 
 def bsa_select_topk(q, k, *, S: int, topk: int, window: int, q_pos0: int = 0, scale: float = 0.0,
@@ -274,6 +288,30 @@ def attn_fwd(q, k, v, q_hat, k_sum, b_sum, idx, *, S: int, window: int, q_pos0: 
     ws, nws = _workspace(p, OP_ATTN_FWD, dev, workspace)
     _raise(lib.hils_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_hat), _ptr(k_sum), _ptr(b_sum),
                              _ptr(idx), _ptr(out), _ptr(lse), _ptr(ws), nws, _stream(dev)))
+    return out, lse
+
+
+def attn_fwd_shat(q, k, v, idx, shat, *, S: int, window: int, q_pos0: int = 0, scale: float = 0.0, out=None,
+                  lse=None):
+    """Eq. 10 prefill from the selection's ids and retrieval scores (select_topk with_shat). q [B,Hq,T,d];
+    k, v [B,Hkv,L,d]; idx [B,Hkv,T,topk] canonical; shat [B,Hq,T,topk] -> out [B,Hq,T,d], lse [B,Hq,T]."""
+    B, Hq, T, d = q.shape
+    Hkv, L = k.shape[1], k.shape[2]
+    topk = idx.shape[-1]
+    dev, dt = q.device, q.dtype
+    for name, t, shape in (("k", k, (B, Hkv, L, d)), ("v", v, (B, Hkv, L, d))):
+        _check(name, t, dt, shape, dev)
+    _check("idx", idx, torch.int32, (B, Hkv, T, topk), dev)
+    _check("shat", shat, torch.float32, (B, Hq, T, topk), dev)
+    if out is None:
+        out = torch.empty((B, Hq, T, d), dtype=dt, device=dev)
+    if lse is None:
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
+    _check("out", out, dt, (B, Hq, T, d), dev)
+    _check("lse", lse, torch.float32, (B, Hq, T), dev)
+    p = make_params(B, T, L, Hq, Hkv, d, S, topk, window, q_pos0, scale, dt)
+    _raise(lib.hils_attn_fwd_shat(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(shat), _ptr(out),
+                                  _ptr(lse), _stream(dev)))
     return out, lse
 
 
@@ -345,11 +383,18 @@ def check(device=None) -> None:
 
 
 def prefill(q, k, v, q_hat, q_land, *, S: int, topk: int, window: int, scale: float = 0.0):
-    """The whole prefill hot path: summaries, selection, attention. Returns (out, lse, idx, k_sum, b_sum)."""
+    """The whole prefill hot path: summaries, selection (with each selected chunk's s^) and attention on
+    those scores; shapes the score-taking attention does not cover use hils_attn_fwd. Returns
+    (out, lse, idx, k_sum, b_sum)."""
     B, Hq, T, d = q.shape
     Hkv, L = k.shape[1], k.shape[2]
     k_sum, b_sum = chunk_summary(k, q_land, S, scale=scale)
-    idx = select_topk(q_hat, k_sum, b_sum, Hkv=Hkv, L=L, S=S, topk=topk, window=window, q_pos0=L - T,
-                          scale=scale)
-    out, lse = attn_fwd(q, k, v, q_hat, k_sum, b_sum, idx, S=S, window=window, q_pos0=L - T, scale=scale)
+    idx, _, shat = select_topk(q_hat, k_sum, b_sum, Hkv=Hkv, L=L, S=S, topk=topk, window=window, q_pos0=L - T,
+                               scale=scale, with_shat=True)
+    try:
+        out, lse = attn_fwd_shat(q, k, v, idx, shat, S=S, window=window, q_pos0=L - T, scale=scale)
+    except HilsError as e:
+        if e.status != 2:  # HILS_ERR_UNSUPPORTED: fall through to the general attention
+            raise
+        out, lse = attn_fwd(q, k, v, q_hat, k_sum, b_sum, idx, S=S, window=window, q_pos0=L - T, scale=scale)
     return out, lse, idx, k_sum, b_sum

@@ -116,25 +116,30 @@ HILS_API hils_status hils_chunk_summary_shared_query(const hils_params *p, const
  * of the group; group score g_c = max_h (s^_{h,c} - LSE_{c'<n} s^_{h,c'}); keep the min(topk, n)
  * largest by (g_c desc, c asc). idx[b,g,i,:] = those ids ascending, then -1.
  * gap (nullable, float32 [B, Hkv, T]) = g_(topk) - g_(topk+1), +inf when n <= topk.
- * Scores in fp32. Supports G * Nc * 4 + next_pow2(Nc) * 8 <= 200 KiB of shared memory per row
- * (Nc <= 8192 at G = 4); longer contexts use hils_decode. Workspace: none.
+ * shat (nullable, float32 [B, Hq, T, topk]): shat[b,h,i,t] = s^_{h, idx[b,g,i,t]} for each head h of
+ * group g, -inf where idx is -1: the retrieval scores hils_attn_fwd_shat takes with idx.
+ * Scores in fp32. On the tensor-core path (bf16, d 128, G <= 4, topk <= 32, 1..128 candidates per row)
+ * the top-k compares keys that keep 16 mantissa bits of g_c, so two candidates whose scores are within
+ * |g_c| * 2^-16 of each other order by chunk id. Otherwise supports G * Nc * 4 + next_pow2(Nc) * 8 <= 200
+ * KiB of shared memory per row (Nc <= 8192 at G = 4); longer contexts use hils_decode. Outputs 16-byte
+ * aligned. Workspace: none.
  */
 HILS_API hils_status hils_select_topk(const hils_params *p, const void *q_hat, const void *k_sum, const float *b_sum,
-                             int32_t *idx, float *gap, void *workspace, size_t workspace_bytes,
+                             int32_t *idx, float *gap, float *shat, void *workspace, size_t workspace_bytes,
                              hils_stream_t stream);
 
 /*
  * hils_select_topk with the Q-Cal projection (Sec. 4) fused into the score kernel: the retrieval query
  * is q^ = q + W_up (W_down q) (rank 32, the token's own query as h, one pair shared by all heads), formed
  * tile by tile in shared memory; no q^ tensor is read or written. q [B, Hq, T, d]; w_down [32, d] and
- * w_up [d, 32] row-major, params.dtype, 16-byte aligned. Outputs, layouts and errors as
- * hils_select_topk. Only the tensor-core shapes (bf16, d 128, G <= 4, topk <= 32, 1..128 candidates per
- * row) and rank 32 are taken (HILS_ERR_UNSUPPORTED otherwise: form q^ and call hils_select_topk).
- * No workspace.
+ * w_up [d, 32] row-major, params.dtype, 16-byte aligned. Outputs (idx, gap, shat), layouts and errors as
+ * hils_select_topk; with shat, a Q-Cal model reaches hils_attn_fwd_shat without ever forming q^.
+ * Only the tensor-core shapes (bf16, d 128, G <= 4, topk <= 32, 1..128 candidates per row) and rank 32
+ * are taken (HILS_ERR_UNSUPPORTED otherwise: form q^ and call hils_select_topk). No workspace.
  */
 HILS_API hils_status hils_select_topk_qcal(const hils_params *p, const void *q, const void *w_down, const void *w_up,
                                            int32_t rank, const void *k_sum, const float *b_sum, int32_t *idx,
-                                           float *gap, hils_stream_t stream);
+                                           float *gap, float *shat, hils_stream_t stream);
 
 /*
  * Naive block-sparse attention selection (Sec. 2), the exact counterpart of hils_select_topk: for every
@@ -166,6 +171,20 @@ HILS_API hils_status hils_bsa_select_topk(const hils_params *p, const void *q, c
 HILS_API hils_status hils_attn_fwd(const hils_params *p, const void *q, const void *k, const void *v, const void *q_hat,
                           const void *k_sum, const float *b_sum, const int32_t *idx, void *out, float *lse,
                           void *workspace, size_t workspace_bytes, hils_stream_t stream);
+
+/*
+ * hils_attn_fwd given the selection's retrieval scores instead of recomputing them: the same Eq. 10
+ * (out, lse) with s^_c read from shat [B, Hq, T, topk] fp32 (slot t of row (b, h, i) scores chunk
+ * idx[b, h/G, i, t], as hils_select_topk writes it). q_hat, k_sum and b_sum are not needed.
+ * idx must be in the canonical form hils_select_topk writes: per row, candidate ids (c < n_p) strictly
+ * ascending, then -1. A row that is not raises a device error word (hils_check then returns
+ * HILS_ERR_INVALID_ARG) and that call's output is invalid; no memory outside the arguments is touched.
+ * Tensor-core shapes only: bf16, d 128, S 64, 128 % G == 0, topk <= 32, at most 8192 chunks
+ * (HILS_ERR_UNSUPPORTED otherwise: call hils_attn_fwd). Pointers 16-byte aligned. No workspace.
+ */
+HILS_API hils_status hils_attn_fwd_shat(const hils_params *p, const void *q, const void *k, const void *v,
+                                        const int32_t *idx, const float *shat, void *out, float *lse,
+                                        hils_stream_t stream);
 
 /*
  * One decode step (stages b-d) for T = M query tokens per sequence at positions q_pos0 .. L-1 with

@@ -55,6 +55,28 @@ def retrieval_group_scores(g: Geometry, q_hat, k_sum, b_sum):
     return f
 
 
+def check_shat(shat: torch.Tensor, idx: torch.Tensor, g: Geometry, q_hat, k_sum, b_sum, what="shat",
+               tol=dict(atol=1e-4, rtol=1e-4)):
+    """Per-head retrieval scores of the selected ids (Eq. 7, fp64 on the given q^ and summaries): slot t of
+    row (b, h, i) holds s^ of chunk idx[b, h/G, i, t], -inf where the id is -1."""
+    sh, ix = np64(shat), idx.cpu().numpy()
+    tau = g.tau()
+    B, Hq, T, K = sh.shape
+    hq = np.arange(Hq)
+    if k_sum.shape[2] == 0:  # no chunk at all: every slot is -1 and scores -inf
+        assert (ix == -1).all() and np.isneginf(sh).all(), f"{what}: slots without a chunk"
+        return
+    for b in range(B):
+        ids = ix[b][hq // g.G]                       # [Hq, T, K]
+        safe = np.where(ids >= 0, ids, 0)
+        kk = k_sum[b][hq[:, None, None], safe]       # [Hq, T, K, d]
+        ref = tau * np.einsum("htd,htkd->htk", q_hat[b], kk) + b_sum[b][hq[:, None, None], safe]
+        ref = np.where(ids >= 0, ref, -np.inf)
+        assert np.array_equal(np.isinf(sh[b]), np.isinf(ref)), f"{what}: -inf slots differ (b {b})"
+        fin = np.isfinite(ref)
+        np.testing.assert_allclose(sh[b][fin], ref[fin], err_msg=f"{what} (b {b})", **tol)
+
+
 def mass_group_scores(g: Geometry, mass):
     """Function (b, kv_group, row) -> group scores from exact chunk masses [B,Hq,T,Nc] (naive BSA, Sec. 2)."""
     _, n = oracle.window(g)

@@ -126,13 +126,13 @@ def test_shared_query_summary_checked():
 
 def test_fused_qcal_rules():
     p = P()
-    st = H.lib.hils_select_topk_qcal(ctypes.byref(p), FAKE, FAKE, FAKE, 16, FAKE, FAKE, FAKE, None, None)
+    st = H.lib.hils_select_topk_qcal(ctypes.byref(p), FAKE, FAKE, FAKE, 16, FAKE, FAKE, FAKE, None, None, None)
     assert st == 2 and b"rank 16" in H.lib.hils_last_error()
     p = P(dtype=1)
-    st = H.lib.hils_select_topk_qcal(ctypes.byref(p), FAKE, FAKE, FAKE, 32, FAKE, FAKE, FAKE, None, None)
+    st = H.lib.hils_select_topk_qcal(ctypes.byref(p), FAKE, FAKE, FAKE, 32, FAKE, FAKE, FAKE, None, None, None)
     assert st == 2 and b"hils_select_topk" in H.lib.hils_last_error()
     p = P()
-    st = H.lib.hils_select_topk_qcal(ctypes.byref(p), FAKE, None, FAKE, 32, FAKE, FAKE, FAKE, None, None)
+    st = H.lib.hils_select_topk_qcal(ctypes.byref(p), FAKE, None, FAKE, 32, FAKE, FAKE, FAKE, None, None, None)
     assert st == 1 and b"w_down is NULL" in H.lib.hils_last_error()
 
 
@@ -152,8 +152,31 @@ def test_bsa_select_rules():
 
 def test_select_too_many_chunks_for_one_cta():
     p = P(T=1, L=1 << 20, q_pos0=(1 << 20) - 1)
-    st = H.lib.hils_select_topk(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, None, 0, None)
+    st = H.lib.hils_select_topk(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, None, None, 0, None)
     assert st == 2 and b"hils_decode" in H.lib.hils_last_error()
+
+
+def test_select_shat_must_be_aligned():
+    p = P()
+    st = H.lib.hils_select_topk(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, ODD, None, 0, None)
+    assert st == 1 and b"shat is not 16-byte aligned" in H.lib.hils_last_error()
+    st = H.lib.hils_select_topk_qcal(ctypes.byref(P(T=128, L=128)), FAKE, FAKE, FAKE, 32, FAKE, FAKE, FAKE, None, ODD,
+                                     None)
+    assert st == 1 and b"shat is not 16-byte aligned" in H.lib.hils_last_error()
+
+
+def attn_shat(p, idx=FAKE, shat=FAKE):
+    return H.lib.hils_attn_fwd_shat(ctypes.byref(p), FAKE, FAKE, FAKE, idx, shat, FAKE, FAKE, None)
+
+
+def test_attn_fwd_shat_rules():
+    """The score-taking attention covers the tensor-core shapes only and checks its pointers on the host."""
+    assert attn_shat(P(dtype=1)) == 2 and b"hils_attn_fwd" in H.lib.hils_last_error()
+    assert attn_shat(P(d=64)) == 2
+    assert attn_shat(P(topk=33)) == 2
+    assert attn_shat(P(Hq=12, Hkv=4)) == 2  # 128 % G != 0
+    assert attn_shat(P(), shat=None) == 1 and b"shat is NULL" in H.lib.hils_last_error()
+    assert attn_shat(P(), idx=ODD) == 1 and b"idx is not 16-byte aligned" in H.lib.hils_last_error()
 
 
 def test_wait_expiry_hook_rejects_limits_before_any_launch():

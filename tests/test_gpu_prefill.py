@@ -6,7 +6,8 @@ import torch
 import oracle
 from oracle import Geometry
 from chunk_wise_hierarchical_summary_b200 import workloads as W
-from tests.parity import BSUM_TOL, TOL, assert_close, check_idx, geometry, np64, retrieval_group_scores, splice
+from tests.parity import (BSUM_TOL, TOL, assert_close, check_idx, check_shat, geometry, np64,
+                           retrieval_group_scores, splice)
 
 pytestmark = pytest.mark.gpu
 
@@ -48,7 +49,37 @@ def run_case(w: W.Workload, seed=0, device="cuda", idx_override=None):
                                            ref["k_sum"], ref["b_sum"], np64(used))
     assert_close(out, ref_out, tol, "out")
     assert_close(lse, ref_lse, tol, "lse")
+    # the selection's retrieval scores of its ids, and the attention that takes them
+    idx2, _, shat = H.select_topk(xd["q_hat"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S, topk=w.topk, window=w.W,
+                                  q_pos0=w.q_pos0, with_shat=True)
+    assert torch.equal(idx2, idx)
+    check_shat(shat, idx, g, np64(x["q_hat"]), np64(k_sum), np64(b_sum))
+    if shat_attention_takes(w):
+        o_s, l_s = H.attn_fwd_shat(xd["q"], xd["k"], xd["v"], idx, shat, S=w.S, window=w.W, q_pos0=w.q_pos0)
+        H.check()
+        gi = idx.cpu().numpy()
+        if near.any():
+            ref_out, ref_lse = oracle.attn_fwd(g, np64(x["q"]), np64(x["k"]), np64(x["v"]), np64(x["q_hat"]),
+                                               ref["k_sum"], ref["b_sum"], gi)
+        assert_close(o_s, ref_out, tol, "out (shat)")
+        assert_close(l_s, ref_lse, tol, "lse (shat)")
+        if gather_attention_is_tc(w):  # same kernel, same scores: the same bits
+            o_g, l_g = H.attn_fwd(xd["q"], xd["k"], xd["v"], xd["q_hat"], k_sum, b_sum, idx, S=w.S, window=w.W,
+                                  q_pos0=w.q_pos0)
+            assert torch.equal(o_s, o_g) and torch.equal(l_s, l_g)
     return dict(near=int(near.sum()), rows=near.size)
+
+
+def shat_attention_takes(w: W.Workload) -> bool:
+    """Shapes hils_attn_fwd_shat covers (the tensor-core attention)."""
+    return w.dtype == "bf16" and w.d == 128 and w.S == 64 and w.topk <= 32 and 128 % w.G == 0
+
+
+def gather_attention_is_tc(w: W.Workload) -> bool:
+    """hils_attn_fwd runs the same tensor-core kernel (its score gather needs G <= 4 and 1..128 candidates)."""
+    last = w.q_pos0 + w.T - 1
+    n_max = max(0, last - w.W + 1) // w.S
+    return shat_attention_takes(w) and w.G <= 4 and 1 <= n_max <= 128
 
 
 def test_tiny_fp32_config():
@@ -76,6 +107,61 @@ def test_tiny_fp32_config():
 ], ids=lambda w: w.name)
 def test_prefill_shapes(w):
     run_case(w)
+
+
+def test_attn_fwd_shat_beyond_128_candidates():
+    """The score-taking attention has no 128-candidate limit: 256 rows at the end of a 12K cache (up to 183
+    candidate chunks, selected by the general kernel with its scores) against the oracle on the GPU's ids."""
+    w = W.Workload("shat_long", B=1, T=256, L=12288, Hq=8, Hkv=2, d=128, S=64, topk=16, W=512, dtype="bf16",
+                   recipe="scaled", q_pos0=12288 - 256)
+    x = W.prefill_inputs(w, seed=21, device="cpu")
+    g = geometry(w)
+    xd = {n: t.cuda() for n, t in x.items()}
+    k_sum, b_sum = H.chunk_summary(xd["k"], xd["q_land"], w.S)
+    ks, bs = np64(k_sum), np64(b_sum)
+    qh = np64(x["q_hat"])
+    idx, gap, shat = H.select_topk(xd["q_hat"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S, topk=w.topk, window=w.W,
+                                   q_pos0=w.q_pos0, with_gap=True, with_shat=True)
+    ridx, rgap = oracle.select_topk(g, qh, ks, bs)
+    check_idx(idx, ridx, rgap, scores=retrieval_group_scores(g, qh, ks, bs))
+    check_shat(shat, idx, g, qh, ks, bs)
+    out, lse = H.attn_fwd_shat(xd["q"], xd["k"], xd["v"], idx, shat, S=w.S, window=w.W, q_pos0=w.q_pos0)
+    H.check()
+    ro, rl = oracle.attn_fwd(g, np64(x["q"]), np64(x["k"]), np64(x["v"]), qh, ks, bs, idx.cpu().numpy())
+    assert_close(out, ro, TOL["bf16"], "out")
+    assert_close(lse, rl, TOL["bf16"], "lse")
+
+
+def test_attn_fwd_shat_flags_non_canonical_ids():
+    """Ids out of order, out of range or repeated are a reported error (HILS_ERR_INVALID_ARG at hils_check),
+    not a fault; the next call with canonical ids is clean and correct."""
+    w = W.Workload("shat_bad", B=1, T=512, L=512, Hq=4, Hkv=1, d=128, S=64, topk=3, W=64, dtype="bf16",
+                   recipe="scaled")
+    x = W.prefill_inputs(w, seed=22, device="cuda")
+    k_sum, b_sum = H.chunk_summary(x["k"], x["q_land"], w.S)
+    idx, _, shat = H.select_topk(x["q_hat"], k_sum, b_sum, Hkv=1, L=w.L, S=w.S, topk=w.topk, window=w.W,
+                                 with_shat=True)
+    good_out, good_lse = H.attn_fwd_shat(x["q"], x["k"], x["v"], idx, shat, S=w.S, window=w.W)
+    H.check()
+    for mutate in ("reverse", "out_of_range", "repeat", "hole"):
+        bad = idx.clone()
+        row = bad[0, 0, 500]
+        assert int((row >= 0).sum()) == 3
+        if mutate == "reverse":
+            bad[0, 0, 500] = row.flip(0)
+        elif mutate == "out_of_range":
+            bad[0, 0, 500, 2] = 10 ** 6
+        elif mutate == "repeat":
+            bad[0, 0, 500, 2] = row[1]
+        else:
+            bad[0, 0, 500, 1] = -1
+        H.attn_fwd_shat(x["q"], x["k"], x["v"], bad, shat, S=w.S, window=w.W)
+        with pytest.raises(H.HilsError, match="canonical") as e:
+            H.check()
+        assert e.value.status == 1
+    out, lse = H.attn_fwd_shat(x["q"], x["k"], x["v"], idx, shat, S=w.S, window=w.W)
+    H.check()
+    assert torch.equal(out, good_out) and torch.equal(lse, good_lse)
 
 
 def test_idx_read_as_a_set():
@@ -143,6 +229,12 @@ def test_prefill_full_size_sampled():
             else:
                 assert_close(out[b:b + 1, hs, rows], ro, tol, "out")
                 assert_close(lse[b:b + 1, hs, rows], rl, tol, "lse")
+    # the bench's path (selection with scores, attention on them) gives the same bits at full size
+    idx_s, _, shat = H.select_topk(x["q_hat"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S, topk=w.topk, window=w.W,
+                                   with_shat=True)
+    out_s, lse_s = H.attn_fwd_shat(x["q"], x["k"], x["v"], idx_s, shat, S=w.S, window=w.W)
+    H.check()
+    assert torch.equal(idx_s, idx) and torch.equal(out_s, out) and torch.equal(lse_s, lse)
     # properties that hold everywhere: every row is finite, ids ascending and candidates only
     assert torch.isfinite(out).all() and torch.isfinite(lse).all()
     pos = torch.arange(w.T, device="cuda")
@@ -206,6 +298,30 @@ def test_select_fused_qcal(w):
     assert near.mean() < 0.25
     finite = np.isfinite(rgap)
     assert_close(gap.cpu().numpy()[finite], rgap[finite], dict(atol=2e-3, rtol=2e-3), "gap")
+
+
+def test_select_fused_qcal_scores_feed_the_attention():
+    """Q-Cal without q^ in memory: the fused selection's scores drive hils_attn_fwd_shat, against the oracle's
+    attention on q^ = bf16(q + W_up W_down q) (the fused kernel rounds q^ to bf16 once) and the GPU's ids."""
+    w = W.Workload("qcal_shat", B=2, T=1000, L=1000, Hq=8, Hkv=2, d=128, S=64, topk=4, W=128, dtype="bf16",
+                   recipe="scaled")
+    x = W.prefill_inputs(w, seed=23)
+    g = geometry(w)
+    xd = {n: t.cuda() for n, t in x.items()}
+    k_sum, b_sum = H.chunk_summary(xd["k"], xd["q_land"], w.S)
+    ks, bs = np64(k_sum), np64(b_sum)
+    idx, _, shat = H.select_topk_qcal(xd["q"], xd["w_down"], xd["w_up"], k_sum, b_sum, Hkv=w.Hkv, L=w.L, S=w.S,
+                                      topk=w.topk, window=w.W, with_shat=True)
+    qhat = oracle.qcal(np64(x["q"]), np64(x["w_down"]), np64(x["w_up"]))
+    qhat_b = np64(torch.from_numpy(qhat).to(torch.bfloat16))
+    ridx, rgap = oracle.select_topk_qcal(g, np64(x["q"]), np64(x["w_down"]), np64(x["w_up"]), ks, bs)
+    check_idx(idx, ridx, rgap, scores=retrieval_group_scores(g, qhat, ks, bs))
+    check_shat(shat, idx, g, qhat_b, ks, bs, tol=dict(atol=2e-3, rtol=2e-3))
+    out, lse = H.attn_fwd_shat(xd["q"], xd["k"], xd["v"], idx, shat, S=w.S, window=w.W)
+    H.check()
+    ro, rl = oracle.attn_fwd(g, np64(x["q"]), np64(x["k"]), np64(x["v"]), qhat_b, ks, bs, idx.cpu().numpy())
+    assert_close(out, ro, TOL["bf16"], "out")
+    assert_close(lse, rl, TOL["bf16"], "lse")
 
 
 def test_select_fused_qcal_full_size_sampled():
