@@ -29,6 +29,7 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kRows = 128;
 constexpr int kStageBytes = 65536;  // q^ tile (32 KiB) + k' tile (32 KiB)
+constexpr int kStages = 3;          // operand stages (heads in flight)
 constexpr int kRank = 32;           // Q-Cal rank of the fused path
 constexpr int kWdRow = 272;         // W_down row (128 bf16) padded: conflict-free fragment loads
 constexpr int kWuRow = 80;          // W_up row (32 bf16) padded
@@ -37,12 +38,12 @@ constexpr int kWuBytes = 128 * kWuRow;
 constexpr int kScoreRow = 129;      // floats per row of exact group scores (odd: conflict-free columns)
 template <int K1MAX>
 constexpr int kListBytes = (kRows * (4 * K1MAX + 1) * 4 + 15) & ~15;
-// Shared memory of the selection: the two operand stages, reused after the MMAs for the per-thread
-// sorted key lists and the exact group scores.
+// Shared memory of the selection: the operand stages, reused after the MMAs for the per-thread sorted
+// key lists, the exact group scores and the staged ids (then the staged scores over the lists).
 template <int K1MAX>
 constexpr size_t select_dyn_smem() {
-    const size_t lists = (size_t)kListBytes<K1MAX> + (size_t)kRows * kScoreRow * 4;
-    return 1024 + (lists > 2 * (size_t)kStageBytes ? lists : 2 * (size_t)kStageBytes);
+    const size_t lists = (size_t)kListBytes<K1MAX> + (size_t)kRows * kScoreRow * 4 + (size_t)kRows * 33 * 4;
+    return 1024 + (lists > kStages * (size_t)kStageBytes ? lists : kStages * (size_t)kStageBytes);
 }
 
 // 32-bit selection key whose ascending order is (score descending, chunk ascending) for chunks < 128:
@@ -129,6 +130,33 @@ __device__ __forceinline__ void qcal_rows(unsigned char *A, const unsigned char 
 
 __device__ unsigned int g_select_tc_errors = 0;
 
+// Explicit shared-space accesses (32-bit shared addresses) for the reused operand stages: their
+// pointers are derived through the alignment arithmetic, and generic accesses there measured slower.
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ float lds_f32(uint32_t a) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ void sts_f32(uint32_t a, float v) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+
+// Orders every later use of v after the preceding tcgen05.wait::ld: the registers pass through an
+// empty volatile asm, which the compiler keeps after the wait and treats as their new definition.
+template <int N>
+__device__ __forceinline__ void reg_fence(float (&v)[N]) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
+}
+
 template <int K1MAX, int GATHER, int QCAL>
 __global__ void __launch_bounds__(kThreads, 1)
 select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, Dims D,
@@ -136,10 +164,11 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
                  float *__restrict__ shat, int *__restrict__ ws_idx, float *__restrict__ ws_shat,
                  const __nv_bfloat16 *__restrict__ w_down, const __nv_bfloat16 *__restrict__ w_up) {
     extern __shared__ unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t tma_bar[2], mma_bar[2], done_bar, qcal_bar[2];
+    __shared__ __align__(8) uint64_t tma_bar[kStages], mma_bar[kStages], qcal_bar[kStages], head_bar[4];
     __shared__ __align__(16) unsigned char wsm[QCAL ? kWdBytes + kWuBytes : 16];
     __shared__ uint32_t s_tmem;
-    __shared__ float bs[4][kRows];
+    __shared__ __align__(16) float bs[4][kRows];   // b' of the group's heads (natural units)
+    __shared__ __align__(16) float bs2[4][kRows];  // b' * log2(e)
     __shared__ float lse[4][kRows];
     __shared__ uint32_t smask[kRows][4];  // selected set of each row (128-bit mask)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -148,7 +177,28 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
     unsigned char *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);  // 1024-byte aligned
     const uint32_t ncols = G == 1 ? 128 : (G == 2 ? 256 : 512);
 
-    if (warp == 0) {
+    // Operand loads start first: per head h the q^ tile [128 rows x 128] and the summary tile
+    // k'_h [128 chunks x 128] (128-byte swizzle) into one of kStages stages.
+    auto load = [&](int hh, int st) {
+        unsigned char *A = base + st * kStageBytes, *Bt = A + 32768;
+        const int hrow = b * D.Hq + g * G + hh;
+        mbar_arrive_expect_tx(&tma_bar[st], kStageBytes);
+        tma_load_2d(A, &qmap, 0, hrow * D.T + i0, &tma_bar[st]);
+        tma_load_2d(A + 16384, &qmap, 64, hrow * D.T + i0, &tma_bar[st]);
+        tma_load_2d(Bt, &kmap, 0, hrow * D.Nc, &tma_bar[st]);
+        tma_load_2d(Bt + 16384, &kmap, 64, hrow * D.Nc, &tma_bar[st]);
+    };
+    if (tid == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&tma_bar[i], 1);
+            mbar_init(&mma_bar[i], 1);
+            mbar_init(&qcal_bar[i], 8);
+        }
+        for (int i = 0; i < 4; ++i) mbar_init(&head_bar[i], 1);
+        fence_mbar_init();
+        for (int hh = 0; hh < G && hh < kStages; ++hh) load(hh, hh);
+    }
+    if (warp == 1) {
         tmem_alloc(&s_tmem, ncols);
         tmem_relinquish();
     }
@@ -159,14 +209,12 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
         *reinterpret_cast<uint4 *>(wsm + (tid >> 4) * kWdRow + (tid & 15) * 16) = wd;
         *reinterpret_cast<uint4 *>(wsm + kWdBytes + (tid >> 2) * kWuRow + (tid & 3) * 16) = wu;
     }
-    if (tid == 32) {
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&tma_bar[i], 1);
-            mbar_init(&mma_bar[i], 1);
-            mbar_init(&qcal_bar[i], 8);
-        }
-        mbar_init(&done_bar, 1);
-        fence_mbar_init();
+    // b' of the group's heads for chunks [0, 128), 0 beyond the summaries.
+    for (int e = tid; e < 4 * kRows; e += blockDim.x) {
+        const int hh = e / kRows, c = e % kRows;
+        const float v = (hh < G && c < D.Nc) ? b_sum[((size_t)b * D.Hq + g * G + hh) * D.Nc + c] : 0.f;
+        bs[hh][c] = v;
+        bs2[hh][c] = v * kLog2e;
     }
     tc_fence_before();
     __syncthreads();
@@ -174,23 +222,16 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
     const uint32_t tmem = s_tmem;
 
     if (warp == 0) {
+        // MMA issuer: D_h = q^_h k'_h^T (M 128, N 128, K 128) into TMEM columns [128h, 128h+128); head_bar[h]
+        // completes when head h's product has landed (every head's bar is committed, also on error paths).
         if (lane == 0) {
-            auto load = [&](int hh, int st) {
-                unsigned char *A = base + st * kStageBytes, *Bt = A + 32768;
-                const int hrow = b * D.Hq + g * G + hh;
-                mbar_arrive_expect_tx(&tma_bar[st], kStageBytes);
-                tma_load_2d(A, &qmap, 0, hrow * D.T + i0, &tma_bar[st]);
-                tma_load_2d(A + 16384, &qmap, 64, hrow * D.T + i0, &tma_bar[st]);
-                tma_load_2d(Bt, &kmap, 0, hrow * D.Nc, &tma_bar[st]);
-                tma_load_2d(Bt + 16384, &kmap, 64, hrow * D.Nc, &tma_bar[st]);
-            };
             bool ok = true;
-            for (int hh = 0; hh < G && hh < 2; ++hh) load(hh, hh);
             const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
-            for (int hh = 0; hh < G && ok; ++hh) {
-                const int st = hh & 1;
+            int hh = 0;
+            for (; hh < G && ok; ++hh) {
+                const int st = hh % kStages;
                 // the tile is ready once TMA has landed it (and, with Q-Cal, warps 8-15 have rewritten it)
-                if (!mbar_wait_bounded(QCAL ? &qcal_bar[st] : &tma_bar[st], (hh >> 1) & 1)) { ok = false; break; }
+                if (!mbar_wait_bounded(QCAL ? &qcal_bar[st] : &tma_bar[st], (hh / kStages) & 1)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t A = smem_u32(base + st * kStageBytes), Bt = A + 32768;
 #pragma unroll
@@ -200,20 +241,21 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
                               ks > 0);
                 }
                 umma_commit(&mma_bar[st]);
-                if (hh + 2 < G) {
-                    if (!mbar_wait_bounded(&mma_bar[st], (hh >> 1) & 1)) { ok = false; break; }
-                    load(hh + 2, st);
+                umma_commit(&head_bar[hh]);
+                if (hh + kStages < G) {
+                    if (!mbar_wait_bounded(&mma_bar[st], (hh / kStages) & 1)) { ok = false; ++hh; break; }
+                    load(hh + kStages, st);
                 }
             }
+            for (; hh < G; ++hh) umma_commit(&head_bar[hh]);  // error path: nothing left waits forever
             if (!ok) atomicOr(&g_select_tc_errors, 1u);
-            umma_commit(&done_bar);  // arrives once every MMA issued above has completed
         }
         __syncwarp();
     } else if (warp >= 8) {
         if constexpr (QCAL != 0) {
             for (int hh = 0; hh < G; ++hh) {
-                const int st = hh & 1;
-                if (!mbar_wait_bounded(&tma_bar[st], (hh >> 1) & 1)) {  // the issuer's wait then expires too
+                const int st = hh % kStages;
+                if (!mbar_wait_bounded(&tma_bar[st], (hh / kStages) & 1)) {  // the issuer's wait then expires too
                     if (lane == 0) atomicOr(&g_select_tc_errors, 4u);
                     break;
                 }
@@ -224,19 +266,12 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
             }
         }
     }
-    // b' of the group's heads for chunks [0, 128), -inf beyond the summaries.
-    for (int e = tid; e < 4 * kRows; e += blockDim.x) {
-        const int hh = e / kRows, c = e % kRows;
-        bs[hh][c] = (hh < G && c < D.Nc) ? b_sum[((size_t)b * D.Hq + g * G + hh) * D.Nc + c] : 0.f;
-    }
-    const bool ok = mbar_wait_bounded(&done_bar, 0);
-    tc_fence_after();
-    __syncthreads();
     const int q = warp & 3, j = warp >> 2;
     const int r = 32 * q + lane;  // tile row = TMEM lane
     const int i = i0 + r;
     const int n_r = (i < D.T) ? window_left(D.q_pos0 + i, D.W, D.S) / D.S : 0;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+    bool ok = true;
 
     if (GATHER) {
         // Gather mode: the caller-given ids of row (query) r are canonicalised once per row (valid ones,
@@ -244,9 +279,11 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
         // memory; then each head's warp writes their retrieval scores s^ = tau D + b' to the workspace.
         // The operand stages are dead once every MMA has completed: [0, 66 KiB) holds the per-thread
         // 33-float rows below, the canonical lists follow.
+        ok = mbar_wait_bounded(&head_bar[G - 1], 0);  // the last product: every MMA has completed
+        tc_fence_after();
+        __syncthreads();
         int *clist = reinterpret_cast<int *>(base + (size_t)kThreads * 33 * sizeof(float));
         int *ccount = clist + kRows * D.topk;
-        const int K = D.topk;
         const bool valid = i < D.T;
         if (j == 0) {
             uint32_t m0 = 0u, m1 = 0u, m2 = 0u, m3 = 0u;
@@ -307,7 +344,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
         }
         tc_fence_before();
         __syncthreads();
-        if (warp == 0) {
+        if (warp == 1) {
             tc_fence_after();
             tmem_dealloc(tmem, ncols);
         }
@@ -315,32 +352,56 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
         return;
     }
 
-    // Phase 1: per-head log-partition over the row's candidates, one 32-column block at a time (block
-    // max, then one rescale of the running sum per block).
+    // Phase 1: per-head log-partition (log2 units) over the row's candidates, starting as soon as the
+    // head's product has landed; one 32-column block at a time (block max, one rescale of the running
+    // sum per block), the next block's TMEM load in flight meanwhile.
     if (j < G) {
         const int hh = j;
+        ok = mbar_wait_bounded(&head_bar[hh], 0);
+        tc_fence_after();
+        const float tau2 = D.tau * kLog2e;
         float m = -INFINITY, z = 0.f;
-#pragma unroll 1
-        for (int t = 0; t < 4; ++t) {
-            float v[32];
-            tmem_ld32(lane_base + hh * 128 + 32 * t, v);
-            tmem_wait_ld();
+        auto block = [&](float (&v)[32], int t) {
+            if (32 * t >= n_r) return;
+            const bool full = 32 * t + 32 <= n_r;
             float bm = -INFINITY;
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-                const int c = 32 * t + e;
-                v[e] = (c < n_r) ? fmaf(D.tau, v[e], bs[hh][c]) * kLog2e : -INFINITY;
-                bm = fmaxf(bm, v[e]);
+                float x = fmaf(tau2, v[e], bs2[hh][32 * t + e]);
+                if (!full) x = (32 * t + e < n_r) ? x : -INFINITY;
+                v[e] = x;
+                bm = fmaxf(bm, x);
             }
             if (bm > -INFINITY) {
                 const float mn = fmaxf(m, bm);
-                float zz = 0.f;
+                float z0 = 0.f, z1 = 0.f;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) zz += ex2_approx(v[e] - mn);
-                z = z * ex2_approx(m - mn) + zz;  // m = -inf at the first block: 2^-inf = 0
+                for (int e = 0; e < 32; e += 2) {
+                    z0 += ex2_approx(v[e] - mn);
+                    z1 += ex2_approx(v[e + 1] - mn);
+                }
+                z = z * ex2_approx(m - mn) + (z0 + z1);  // m = -inf at the first block: 2^-inf = 0
                 m = mn;
             }
-        }
+        };
+        const uint32_t col = lane_base + hh * 128;
+        float va[32], vb[32];
+        tmem_ld32(col, va);
+        tmem_wait_ld();
+        reg_fence(va);
+        tmem_ld32(col + 32, vb);
+        block(va, 0);
+        tmem_wait_ld();
+        reg_fence(vb);
+        tmem_ld32(col + 64, va);
+        block(vb, 1);
+        tmem_wait_ld();
+        reg_fence(va);
+        tmem_ld32(col + 96, vb);
+        block(va, 2);
+        tmem_wait_ld();
+        reg_fence(vb);
+        block(vb, 3);
         lse[hh][r] = (n_r > 0) ? (m + log2f(z)) * kLn2 : 0.f;
     }
     tc_fence_before();
@@ -351,123 +412,168 @@ select_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
     // registers; the exact scores go to shared memory for the gap. The operand stages are dead once every
     // MMA has completed: [0, list bytes) holds the lists, the score rows follow.
     constexpr int kRowKeys = 4 * K1MAX + 1;  // odd: neighbouring rows' lists fall in different banks
-    uint32_t *lists = reinterpret_cast<uint32_t *>(base);
-    float *gsc = reinterpret_cast<float *>(base + kListBytes<K1MAX>);  // [kRows][kScoreRow]
+    const uint32_t lists = smem_u32(base);                        // uint32 [kRows][kRowKeys]
+    const uint32_t gsc = lists + kListBytes<K1MAX>;               // float [kRows][kScoreRow]
     {
         uint32_t key[32];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
             const int cb = 32 * j + 16 * half;  // first column of this 16-wide piece
+            float v[4][16];
+#pragma unroll
+            for (int hh = 0; hh < 4; ++hh)
+                if (hh < G) tmem_ld16(lane_base + hh * 128 + cb, v[hh]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int hh = 0; hh < 4; ++hh) reg_fence(v[hh]);
             float gv[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) gv[e] = -INFINITY;
-            for (int hh = 0; hh < G; ++hh) {
-                float v[16];
-                tmem_ld16(lane_base + hh * 128 + cb, v);
-                tmem_wait_ld();
-                const float l = lse[hh][r];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) gv[e] = fmaxf(gv[e], fmaf(D.tau, v[e], bs[hh][cb + e]) - l);
+            for (int hh = 0; hh < 4; ++hh) {
+                if (hh < G) {
+                    const float l = lse[hh][r];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) gv[e] = fmaxf(gv[e], fmaf(D.tau, v[hh][e], bs[hh][cb + e]) - l);
+                }
             }
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const int c = cb + e;
                 key[16 * half + e] = (c < n_r) ? sel_key32(gv[e], (uint32_t)c) : 0xffffffffu;
-                gsc[r * kScoreRow + c] = gv[e];
+                sts_f32(gsc + 4 * (r * kScoreRow + c), gv[e]);
             }
         }
         sort32_u32(key);
 #pragma unroll
-        for (int t = 0; t < K1MAX; ++t) lists[r * kRowKeys + j * K1MAX + t] = t < 32 ? key[t] : 0xffffffffu;
+        for (int t = 0; t < K1MAX; ++t) sts_u32(lists + 4 * (r * kRowKeys + j * K1MAX + t), t < 32 ? key[t] : 0xffffffffu);
     }
-    tc_fence_before();
     __syncthreads();
 
-    // Phase 3: one thread per row merges its four sorted lists: the first min(K + 1, n) keys give the
-    // selected set (a 128-bit mask, read out ascending) and the k-th and (k+1)-th ids for the gap.
-    if (tid < kRows) {
-        const int rr = tid, ii = i0 + rr;
-        uint32_t m0 = 0u, m1 = 0u, m2 = 0u, m3 = 0u;
-        if (ii < D.T) {
-            const int nn = window_left(D.q_pos0 + ii, D.W, D.S) / D.S;
-            const uint32_t *Lr = lists + rr * kRowKeys;
-            int p0 = 0, p1 = 0, p2 = 0, p3 = 0;
-            const int need = min(K + 1, nn);
-            int ck = 0, ck1 = 0;
-            for (int t = 0; t < need; ++t) {
-                const uint32_t a0 = p0 < K1MAX ? Lr[p0] : 0xffffffffu, a1 = p1 < K1MAX ? Lr[K1MAX + p1] : 0xffffffffu;
-                const uint32_t a2 = p2 < K1MAX ? Lr[2 * K1MAX + p2] : 0xffffffffu;
-                const uint32_t a3 = p3 < K1MAX ? Lr[3 * K1MAX + p3] : 0xffffffffu;
-                const uint32_t mm = min(min(a0, a1), min(a2, a3));
-                if (mm == a0) ++p0;
-                else if (mm == a1) ++p1;
-                else if (mm == a2) ++p2;
-                else ++p3;
-                const int c = (int)(mm & 127u);
-                if (t < K) {
-                    const uint32_t bit = 1u << (c & 31);
-                    const int w = c >> 5;
-                    m0 |= (w == 0) ? bit : 0u;
-                    m1 |= (w == 1) ? bit : 0u;
-                    m2 |= (w == 2) ? bit : 0u;
-                    m3 |= (w == 3) ? bit : 0u;
-                }
-                if (t == K - 1) ck = c;
-                if (t == K) ck1 = c;
-            }
-            int *row = idx + (((size_t)b * D.Hkv + g) * D.T + ii) * K;
-            int ns = 0;
-            const uint32_t words[4] = {m0, m1, m2, m3};
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                uint32_t x = words[w];
-                while (x) {
-                    row[ns++] = 32 * w + __ffs(x) - 1;
-                    x &= x - 1u;
+    // Phase 3: the four sorted lists of a row are merged by four lanes of one warp (warp w takes rows
+    // 8w .. 8w+7, lane 4u + l holds the head of list l of row 8w + u): per step the row's minimum by two
+    // shuffles, the owning lane records it and loads its next key. The first min(K + 1, n) keys give the
+    // selected set (a 128-bit mask, one word per lane, read out ascending) and the k-th and (k+1)-th ids
+    // for the gap. Ids and scores are staged in shared memory (rows of K + 1 words, conflict-free) and
+    // leave in one coalesced copy per tensor: the CTA's rows are contiguous.
+    const int KP = K + 1;
+    const uint32_t sidx = gsc + kRows * kScoreRow * 4;  // int [kRows][KP]
+    const uint32_t sshat = lists;                       // float [G][kRows][KP], once the lists are dead
+    {
+        const int rr = 8 * warp + (lane >> 2), l = lane & 3;
+        const int ii = i0 + rr;
+        const int nn = ii < D.T ? window_left(D.q_pos0 + ii, D.W, D.S) / D.S : 0;
+        const int need = min(K + 1, nn);
+        const uint32_t Lp = lists + 4 * (rr * kRowKeys + l * K1MAX);
+        uint32_t a = lds_u32(Lp);
+        int p = 1;
+        uint32_t word = 0u;  // selected ids c with c >> 5 == l
+        uint32_t kk = 0u, kk1 = 0u;
+        const int steps = __reduce_max_sync(0xffffffffu, need);
+        for (int t = 0; t < steps; ++t) {
+            uint32_t m = min(a, __shfl_xor_sync(0xffffffffu, a, 1));
+            m = min(m, __shfl_xor_sync(0xffffffffu, m, 2));
+            if (t < need) {
+                const uint32_t c = m & 127u;
+                if (t < K && (int)(c >> 5) == l) word |= 1u << (c & 31);
+                if (t == K - 1) kk = c;
+                if (t == K) kk1 = c;
+                if (a == m) {
+                    a = p < K1MAX ? lds_u32(Lp + 4 * p) : 0xffffffffu;
+                    ++p;
                 }
             }
-            for (int t = ns; t < K; ++t) row[t] = -1;
-            if (gap)
-                gap[((size_t)b * D.Hkv + g) * D.T + ii] =
-                    (nn > K) ? gsc[rr * kScoreRow + ck] - gsc[rr * kScoreRow + ck1] : INFINITY;
         }
-        smask[rr][0] = m0;
-        smask[rr][1] = m1;
-        smask[rr][2] = m2;
-        smask[rr][3] = m3;
+        // ids of word l go to slots [popc of the lower words, ...); the rest of the row is -1
+        const int g4 = lane & ~3;
+        const uint32_t w0 = __shfl_sync(0xffffffffu, word, g4), w1 = __shfl_sync(0xffffffffu, word, g4 | 1),
+                       w2 = __shfl_sync(0xffffffffu, word, g4 | 2), w3 = __shfl_sync(0xffffffffu, word, g4 | 3);
+        if (ii < D.T) {
+            const int before = (l > 0 ? __popc(w0) : 0) + (l > 1 ? __popc(w1) : 0) + (l > 2 ? __popc(w2) : 0);
+            const int total = __popc(w0) + __popc(w1) + __popc(w2) + __popc(w3);
+            const uint32_t row = sidx + 4 * rr * KP;
+            int u = before;
+            for (uint32_t x = word; x; x &= x - 1u) sts_u32(row + 4 * u++, 32 * l + __ffs(x) - 1);
+            if (l == 3)
+                for (int t = total; t < K; ++t) sts_u32(row + 4 * t, 0xffffffffu);
+            if (gap && l == 0)
+                gap[((size_t)b * D.Hkv + g) * D.T + ii] =
+                    (nn > K) ? lds_f32(gsc + 4 * (rr * kScoreRow + kk)) - lds_f32(gsc + 4 * (rr * kScoreRow + kk1))
+                             : INFINITY;
+        } else {
+            word = 0u;
+        }
+        smask[rr][l] = word;
     }
 
     // Phase 4 (optional): each head's retrieval score s^ = tau D + b' of the selected ids, in id order,
-    // -inf in the unused slots.
+    // -inf in the unused slots. Thread (row, block j) writes the selected columns of its 32-column block
+    // for every head (slot = selected ids before it), the next head's TMEM load in flight meanwhile.
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
     if (shat != nullptr) {
-        __syncthreads();
-        if (j < G) {  // warp-uniform: every lane executes the TMEM loads
-            const int hh = j;
-            float *dst = shat + (((size_t)b * D.Hq + g * G + hh) * D.T + (i < D.T ? i : 0)) * K;
-            int u = 0;
-#pragma unroll 1
-            for (int t = 0; t < 4; ++t) {
-                float v[32];
-                tmem_ld32(lane_base + hh * 128 + 32 * t, v);
-                tmem_wait_ld();
-                const uint32_t m = smask[r][t];
-                if (i < D.T) {
+        const uint32_t w0 = smask[r][0], w1 = smask[r][1], w2 = smask[r][2], w3 = smask[r][3];
+        const uint32_t mj = j == 0 ? w0 : (j == 1 ? w1 : (j == 2 ? w2 : w3));
+        const int before = (j > 0 ? __popc(w0) : 0) + (j > 1 ? __popc(w1) : 0) + (j > 2 ? __popc(w2) : 0);
+        const int total = __popc(w0) + __popc(w1) + __popc(w2) + __popc(w3);
+        const bool valid = i < D.T;
+        auto emit = [&](const float (&v)[32], int hh) {
+            if (!valid) return;
+            const uint32_t dst = sshat + 4 * (hh * kRows + r) * KP;
+            int u = before;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if ((m >> e) & 1u) dst[u++] = fmaf(D.tau, v[e], bs[hh][32 * t + e]);
-                }
-            }
-            if (i < D.T)
-                for (int t = u; t < K; ++t) dst[t] = -INFINITY;
+            for (int e = 0; e < 32; ++e)
+                if ((mj >> e) & 1u) sts_f32(dst + 4 * u++, fmaf(D.tau, v[e], bs[hh][32 * j + e]));
+            if (j == 3)
+                for (int t = total; t < K; ++t) sts_f32(dst + 4 * t, -INFINITY);
+        };
+        const uint32_t col = lane_base + 32 * j;
+        float va[32], vb[32];
+        tmem_ld32(col, va);
+        tmem_wait_ld();
+        reg_fence(va);
+        if (G > 1) tmem_ld32(col + 128, vb);
+        emit(va, 0);
+        if (G > 1) {
+            tmem_wait_ld();
+            reg_fence(vb);
+            if (G > 2) tmem_ld32(col + 256, va);
+            emit(vb, 1);
+        }
+        if (G > 2) {
+            tmem_wait_ld();
+            reg_fence(va);
+            if (G > 3) tmem_ld32(col + 384, vb);
+            emit(va, 2);
+        }
+        if (G > 3) {
+            tmem_wait_ld();
+            reg_fence(vb);
+            emit(vb, 3);
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, ncols);
     }
-    if (!ok && tid == 0) atomicOr(&g_select_tc_errors, 2u);
+    // coalesced copies out: lane = slot, warps stride over the rows
+    const int nr = min(kRows, D.T - i0);
+    if (lane < K) {
+        int *gidx = idx + (((size_t)b * D.Hkv + g) * D.T + i0) * K;
+        for (int rr = warp; rr < nr; rr += kThreads / 32)
+            gidx[rr * K + lane] = (int)lds_u32(sidx + 4 * (rr * KP + lane));
+        if (shat != nullptr) {
+            for (int hh = 0; hh < G; ++hh) {
+                float *gs = shat + (((size_t)b * D.Hq + g * G + hh) * D.T + i0) * K;
+                const uint32_t ss = sshat + 4 * hh * kRows * KP;
+                for (int rr = warp; rr < nr; rr += kThreads / 32) gs[rr * K + lane] = lds_f32(ss + 4 * (rr * KP + lane));
+            }
+        }
+    }
+    if (!ok) atomicOr(&g_select_tc_errors, 2u);
 }
 
 }  // namespace
@@ -543,7 +649,7 @@ cudaError_t launch_gather_shat_tc(const Dims &D, const void *q_hat, const void *
         !make_tmap_bf16_2d(&kmap, k_sum, (uint64_t)D.B * D.Hq * D.Nc, 128, 128, 128))
         return cudaErrorInvalidValue;
     dim3 grid((D.T + kRows - 1) / kRows, D.Hkv, D.B);
-    const size_t smem = 1024 + 2 * (size_t)kStageBytes;
+    const size_t smem = select_dyn_smem<17>();
     cudaFuncSetAttribute(select_tc_kernel<17, 1, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     select_tc_kernel<17, 1, 0><<<grid, kThreads, smem, stream>>>(qmap, kmap, D, b_sum, const_cast<int *>(idx), nullptr,
                                                                   nullptr, ws_idx, ws_shat, nullptr, nullptr);
