@@ -8,9 +8,10 @@
 //              (max, sum exp) of each slice. This launch streams the decode step's dominant bytes.
 //  2. select   per (b, KV group): per-head LSE folded from the partials, group score
 //              g_c = max_h (s^_{h,c} - LSE_h) as 64-bit keys (score desc, chunk id asc), top-k. For
-//              topk <= 32 and G <= 8 one CTA per group: each warp sorts batches of 256 keys in registers
-//              and merges their best 32 into a running top-32, then the warps' lists are reduced in
-//              the CTA. Otherwise several CTAs per group keep their part's top-k and the last CTA to
+//              topk <= 32 and G <= 8 one CTA per group: up to 2048 candidates, each of eight warps sorts
+//              its 256 keys in registers and warp 0 merges their best 32; longer lists keep an exact
+//              lower bound of the top-k and sort the few candidates at or below it. With few groups and
+//              very long lists several CTAs per group keep their part's top-k and the last CTA to
 //              finish (atomic counter, no waiting) merges them.
 //  3. attend   bf16 d 128 S 64 G <= 8: decode_attn_mma.cu (split-K CTAs over the group's tiles,
 //              warp-level MMAs, online Eq. 10 merge). Otherwise here: one S-token tile (a selected
@@ -691,6 +692,111 @@ decode_select_warp_kernel(Dims D, DecodePlan P, const float *__restrict__ scores
     }
 }
 
+// Short candidate lists (n <= 2048, topk <= 32, G <= GM): one CTA of eight warps per (b, KV group, query)
+// with every memory read issued up front. Warp w holds candidates [256w, 256w + 256), eight a lane; the
+// per-head LSE is folded from the score kernel's slice partials as in the kernel above; each warp sorts
+// its 256 keys in registers and keeps the best 32, and warp 0 merges the warps' lists. Same keys as the
+// kernel above (group score desc, chunk id asc), so the same ids; about a third of its latency on short
+// lists, whose cost was its phases' barriers and round trips rather than the candidates.
+constexpr int kSelSThreads = 256;
+constexpr int kSelSNpl = 8;
+constexpr int kSelSMax = kSelSThreads * kSelSNpl;
+
+template <int GM>
+__global__ void __launch_bounds__(kSelSThreads, 1)
+decode_select_short_kernel(Dims D, DecodePlan P, const float *__restrict__ scores, const float *__restrict__ part,
+                           int *__restrict__ sel, int *__restrict__ idx_out) {
+    __shared__ float lse[8];
+    __shared__ __align__(8) uint64_t lists[kSelSThreads / 32][32];
+    const int g = blockIdx.x, M = D.T, b = blockIdx.y / M, m = blockIdx.y % M;
+    const int G = D.G, K = D.topk;
+    const int n = window_left(D.q_pos0 + m, D.W, D.S) / D.S;
+    const size_t bgm = ((size_t)b * D.Hkv + g) * M + m;
+    // the attention grid may start now: its CTAs load and fold their window tiles while this grid selects
+    grid_dep_launch();
+    grid_dep_wait();  // the score grid's scores and partials
+    const size_t hs = (size_t)M * P.n;  // stride between the group's heads in the score rows
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int *out = sel + bgm * K;
+    int *out2 = idx_out ? idx_out + bgm * K : nullptr;
+    if (n == 0) {
+        for (int t = tid; t < K; t += blockDim.x) {
+            out[t] = -1;
+            if (out2) out2[t] = -1;
+        }
+        return;
+    }
+    const float *sc0 = scores + (((size_t)b * D.Hq + g * G) * M + m) * P.n;
+    float raw[GM][kSelSNpl];
+#pragma unroll
+    for (int hh = 0; hh < GM; ++hh)
+#pragma unroll
+        for (int i = 0; i < kSelSNpl; ++i) {
+            const int c = warp * 32 * kSelSNpl + i * 32 + lane;
+            raw[hh][i] = (hh < G && c < n) ? sc0[hh * hs + c] : -INFINITY;
+        }
+    if (warp < G) {
+        const int hh = warp;
+        const int np = P.nslices * kScorePartsPerSliceHost;
+        const float2 *ph = reinterpret_cast<const float2 *>(part + (((size_t)b * D.Hq + g * G + hh) * M + m) * np * 2);
+        float Mx = -INFINITY, Z = 0.f;
+        for (int s0 = 0; s0 < np; s0 += 32 * 8) {
+            float2 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int si = s0 + u * 32 + lane;
+                v[u] = (si < np) ? ph[si] : make_float2(-INFINITY, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (v[u].x > Mx) {
+                    Z = Z * __expf(Mx - v[u].x) + v[u].y;
+                    Mx = v[u].x;
+                } else if (v[u].x > -INFINITY) {
+                    Z += v[u].y * __expf(v[u].x - Mx);
+                }
+            }
+        }
+        const float MM = warp_max(Mx);
+        Z = (Mx > -INFINITY) ? Z * __expf(Mx - MM) : 0.f;
+        Z = warp_sum(Z);
+        if (lane == 0) lse[hh] = MM + logf(Z);
+    }
+    __syncthreads();
+    float L[GM];
+#pragma unroll
+    for (int hh = 0; hh < GM; ++hh) L[hh] = hh < G ? lse[hh] : 0.f;
+    uint64_t kv[kSelSNpl];
+#pragma unroll
+    for (int i = 0; i < kSelSNpl; ++i) {
+        const int c = warp * 32 * kSelSNpl + i * 32 + lane;
+        float gv = -INFINITY;
+#pragma unroll
+        for (int hh = 0; hh < GM; ++hh)
+            if (hh < G) gv = fmaxf(gv, raw[hh][i] - L[hh]);
+        kv[i] = (c < n) ? desc_value_key(gv, (uint32_t)c) : ~0ull;
+    }
+    const int nwarps = (n + 32 * kSelSNpl - 1) / (32 * kSelSNpl);  // warps holding candidates
+    if (warp < nwarps) {
+        warp_bitonic_sort<kSelSNpl>(kv);
+        lists[warp][lane] = warp_first32<kSelSNpl>(kv);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        uint64_t top = lists[0][lane];
+        for (int w = 1; w < nwarps; ++w) top = warp_merge_lowest32(top, lists[w][lane]);
+        // the selected ids (first min(K, n) keys), written ascending, -1 padded
+        const int kk = min(K, n);
+        uint64_t ids[1] = {(lane < kk && top != ~0ull) ? (uint64_t)desc_key_index(top) : ~0ull};
+        warp_bitonic_sort<1>(ids);
+        if (lane < K) {
+            const int v = ids[0] == ~0ull ? -1 : (int)ids[0];
+            out[lane] = v;
+            if (out2) out2[lane] = v;
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------- 3. attend (+ combine)
 
 template <typename T, int DPL>
@@ -932,7 +1038,13 @@ cudaError_t launch_t(const Dims &D, const void *q, const void *q_hat, const void
     // (Measured at B1: 8184 candidates faster on one CTA, 16376 and more faster split.)
     const bool wide = D.T == 1 && D.B * D.Hkv < 32 && P.n >= 12288 && next_pow2(P.nparts * D.topk) <= kSelMerge;
     cudaError_t es;
-    if (!wide && D.topk <= 32 && D.G <= 4)
+    if (!wide && D.topk <= 32 && P.n <= kSelSMax && D.G <= 4)
+        es = launch_pdl(decode_select_short_kernel<4>, dim3(D.Hkv, D.B * D.T), dim3(kSelSThreads), 0, stream, D, P,
+                        (const float *)scores, (const float *)part, sel, idx_out);
+    else if (!wide && D.topk <= 32 && P.n <= kSelSMax && D.G <= 8)
+        es = launch_pdl(decode_select_short_kernel<8>, dim3(D.Hkv, D.B * D.T), dim3(kSelSThreads), 0, stream, D, P,
+                        (const float *)scores, (const float *)part, sel, idx_out);
+    else if (!wide && D.topk <= 32 && D.G <= 4)
         es = launch_pdl(decode_select_warp_kernel<4>, dim3(D.Hkv, D.B * D.T), dim3(kSelWThreads), 0, stream, D, P,
                         (const float *)scores, (const float *)part, sel, idx_out);
     else if (!wide && D.topk <= 32 && D.G <= 8)

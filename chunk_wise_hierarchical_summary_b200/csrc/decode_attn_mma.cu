@@ -40,6 +40,7 @@ constexpr uint32_t kQRowBytes = 272;
 constexpr int kPStride = 72;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kPartStride = 132;  // floats per (head, split) partial: M, l, 2 pad, o[128] (16-byte aligned)
+constexpr int kMaxSplits = 16;    // CTAs per (b, KV group, query)
 
 __device__ unsigned int g_decode_attn_errors = 0;
 
@@ -107,20 +108,24 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     auto append_selected = [&]() {
         grid_dep_wait();  // the selection grid's ids (and, through it, the scores)
         __syncthreads();  // every thread is past its pre-wait tiles before the list grows
-        if (tid == 0) {
+        if (warp == 0) {
+            // this CTA's selected slots t0, t0 + nsplit, ... read 32 at a time, one per lane, in order
             int n2 = nw;
-            for (int t = split + ((wt - split + nsplit - 1) / nsplit) * nsplit; t < ntiles && n2 < kMaxTiles;
-                 t += nsplit) {
-                if (t < wt) continue;
-                const int c = sel[bgm * K + (t - wt)];
-                if (c < 0) continue;
-                Tile tl;
-                tl.j0 = c * S;
-                tl.jn = S;
-                tl.c = c;
-                tiles[n2++] = tl;
+            for (int t = split + ((wt - split + nsplit - 1) / nsplit) * nsplit + lane * nsplit;
+                 __any_sync(0xffffffffu, t < ntiles); t += 32 * nsplit) {
+                const int c = (t < ntiles && t >= wt) ? sel[bgm * K + (t - wt)] : -1;
+                const unsigned take = __ballot_sync(0xffffffffu, c >= 0);
+                const int at = n2 + __popc(take & ((1u << lane) - 1u));
+                if (c >= 0 && at < kMaxTiles) {
+                    Tile tl;
+                    tl.j0 = c * S;
+                    tl.jn = S;
+                    tl.c = c;
+                    tiles[at] = tl;
+                }
+                n2 += __popc(take);
             }
-            s_nt = n2;
+            if (lane == 0) s_nt = min(n2, kMaxTiles);
         }
         __syncthreads();
         nt = s_nt;
@@ -317,20 +322,25 @@ decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     for (int hh = warp; hh < G; hh += blockDim.x >> 5) {
         const size_t hr = ((size_t)b * D.Hq + g * G + hh) * M + m;
         const float *ph = partial + hr * nsplit * kPartStride;
+        // every load of the head's partials in flight at once (nsplit <= kMaxSplits)
         const float ms = lane < nsplit ? __ldcg(ph + (size_t)lane * kPartStride) : -INFINITY;
         const float ls = lane < nsplit ? __ldcg(ph + (size_t)lane * kPartStride + 1) : 0.f;
+        float4 v4[kMaxSplits];
+#pragma unroll
+        for (int s2 = 0; s2 < kMaxSplits; ++s2)
+            v4[s2] = s2 < nsplit ? __ldcg(reinterpret_cast<const float4 *>(ph + (size_t)s2 * kPartStride + 4) + lane)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
         const float Mx = warp_max(ms);
         const float rs = ms == -INFINITY ? 0.f : ex2_approx(ms - Mx);  // a CTA with no tiles has weight 0
         const float Z = warp_sum(ls * rs);
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-        for (int s2 = 0; s2 < nsplit; ++s2) {
-            const float r = __shfl_sync(0xffffffffu, rs, s2);
-            const float4 v4 = __ldcg(reinterpret_cast<const float4 *>(ph + (size_t)s2 * kPartStride + 4) + lane);
-            acc[0] = fmaf(v4.x, r, acc[0]);
-            acc[1] = fmaf(v4.y, r, acc[1]);
-            acc[2] = fmaf(v4.z, r, acc[2]);
-            acc[3] = fmaf(v4.w, r, acc[3]);
+#pragma unroll
+        for (int s2 = 0; s2 < kMaxSplits; ++s2) {
+            const float r = __shfl_sync(0xffffffffu, rs, s2);  // 0 for s2 >= nsplit (ms = -inf there)
+            acc[0] = fmaf(v4[s2].x, r, acc[0]);
+            acc[1] = fmaf(v4[s2].y, r, acc[1]);
+            acc[2] = fmaf(v4[s2].z, r, acc[2]);
+            acc[3] = fmaf(v4[s2].w, r, acc[3]);
         }
         const float inv = Z > 0.f ? 1.f / Z : 0.f;
         const __nv_bfloat162 h01 = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
@@ -355,7 +365,7 @@ bool decode_attn_mma_supported(const Dims &D, int dtype, const void *q, const vo
 // most 16 (so the last CTA merges few partials: at small batches a split is then 2-3 tiles).
 int decode_attn_mma_splits(const Dims &D, int ntiles) {
     const int per_bg = std::max(1, (kCtasPerSm * num_sms()) / std::max(1, D.B * D.Hkv * D.T));
-    return std::max(1, std::min(std::min(per_bg, ntiles), 16));
+    return std::max(1, std::min(std::min(per_bg, ntiles), kMaxSplits));
 }
 
 unsigned int decode_attn_mma_error_flags(bool clear) {
