@@ -531,6 +531,7 @@ decode_select_warp_kernel(Dims D, DecodePlan P, const float *__restrict__ scores
     __shared__ float lse[8];
     __shared__ __align__(8) uint64_t keys[kSelWThreads];
     __shared__ __align__(8) uint64_t surv[kSelWCap];
+    __shared__ int sel_ids[32];
     __shared__ uint64_t s_bound;
     __shared__ int s_count;
     // grid (Hkv, B * M): query m of sequence b; its candidates are the chunks before its window
@@ -664,24 +665,36 @@ decode_select_warp_kernel(Dims D, DecodePlan P, const float *__restrict__ scores
     }
     __syncthreads();
     const int count = s_count;
-    uint64_t top = ~0ull;  // warp 0: the selection's keys, ascending, one per lane
+    const int kk = min(K, n);
     if (count <= kSelWCap) {
-        if (warp == 0) {
-            uint64_t kv[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int e = lane * 4 + i;
-                kv[i] = e < count ? surv[e] : ~0ull;
-            }
-            warp_bitonic_sort<4>(kv);
-            top = warp_first32<4>(kv);
+        // The keys are distinct: a survivor's rank is the number of smaller survivors (one thread each,
+        // every read a shared-memory broadcast). The kk best go to sel_ids in score order; then each of
+        // those ids is ranked among them and written in ascending order.
+        if (tid < count) {
+            const uint64_t k = surv[tid];
+            int rank = 0;
+            for (int j = 0; j < count; ++j) rank += surv[j] < k ? 1 : 0;
+            if (rank < kk) sel_ids[rank] = (int)desc_key_index(k);
         }
-    } else {
-        top = select_tied_fallback<GM>(sc0, hs, G, n, rounds, L, keys);
+        __syncthreads();
+        if (tid < K) {
+            int v = -1;
+            if (tid < kk) {
+                const int id = sel_ids[tid];
+                int r2 = 0;
+                for (int j = 0; j < kk; ++j) r2 += sel_ids[j] < id ? 1 : 0;
+                out[r2] = id;
+                if (out2) out2[r2] = id;
+            } else {
+                out[tid] = v;
+                if (out2) out2[tid] = v;
+            }
+        }
+        return;
     }
+    uint64_t top = select_tied_fallback<GM>(sc0, hs, G, n, rounds, L, keys);  // warp 0: keys ascending
     if (warp == 0) {
-        // the selected ids (first min(K, n) keys), written ascending, -1 padded
-        const int kk = min(K, n);
+        // the selected ids (first kk keys), written ascending, -1 padded
         uint64_t ids[1] = {(lane < kk && top != ~0ull) ? (uint64_t)desc_key_index(top) : ~0ull};
         warp_bitonic_sort<1>(ids);
         if (lane < K) {

@@ -40,7 +40,7 @@ constexpr uint32_t kQRowBytes = 272;
 constexpr int kPStride = 72;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kPartStride = 132;  // floats per (head, split) partial: M, l, 2 pad, o[128] (16-byte aligned)
-constexpr int kMaxSplits = 16;    // CTAs per (b, KV group, query)
+constexpr int kMaxSplits = 32;    // CTAs per (b, KV group, query)
 
 __device__ unsigned int g_decode_attn_errors = 0;
 
