@@ -26,10 +26,12 @@ bool make_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64
 
 namespace {
 
-constexpr int kStages = 3;
+// Two stages and five CTAs per SM (more consumer warps per SM) beat three stages at three CTAs: the
+// per-tile chain of the consumers, not the copies in flight, bounds the stream.
+constexpr int kStages = 2;
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
-constexpr int kCtasPerSm = 3;
+constexpr int kCtasPerSm = 5;
 constexpr uint32_t kKBytes = 16384;      // 64 keys x 128 columns bf16
 constexpr uint32_t kQRowBytes = 272;     // one landmark row (256 B) padded: conflict-free fragment reads
 constexpr uint32_t kQBytes = 8 * kQRowBytes;
