@@ -67,6 +67,14 @@ def check_group_rows(w, x, out, lse, idx, groups):
                recipe="needle", q_pos0=4999, needles=5),
     W.Workload("dec_g1", B=1, T=1, L=3000, Hq=3, Hkv=3, d=128, S=64, topk=8, W=200, dtype="bf16",
                recipe="needle", q_pos0=2999, needles=3),
+    # the selection kernels' boundary: 2048 candidates (the short-list kernel, every warp full, G = 8) and
+    # 2049 (the bounded survivor kernel with its parallel ranking, G = 4 and G = 8)
+    W.Workload("dec_short_list_full_g8", B=1, T=1, L=131584, Hq=8, Hkv=1, d=128, S=64, topk=32, W=512,
+               dtype="bf16", recipe="needle", q_pos0=131583, needles=4),
+    W.Workload("dec_long_list_first_g4", B=1, T=1, L=131648, Hq=4, Hkv=1, d=128, S=64, topk=32, W=512,
+               dtype="bf16", recipe="needle", q_pos0=131647, needles=4),
+    W.Workload("dec_long_list_first_g8", B=1, T=1, L=131648, Hq=8, Hkv=1, d=128, S=64, topk=16, W=512,
+               dtype="bf16", recipe="needle", q_pos0=131647, needles=4),
     # one KV group over a 1M-token cache (16385 candidates): the list is split over several selection CTAs
     W.Workload("dec_long_one_group", B=1, T=1, L=1049176, Hq=4, Hkv=1, d=128, S=64, topk=8, W=512, dtype="bf16",
                recipe="needle", q_pos0=1049175, needles=4),
