@@ -172,8 +172,10 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
     __shared__ float lsh[128][kMaxK];  // per row: the matching s^ in log2 units
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = D.G, QT = 128 / G;
-    // late query tiles visit the most chunks: launch them first (short CTAs make the grid's tail)
-    const int i0 = (gridDim.x - 1 - blockIdx.x) * QT, g = blockIdx.y, b = blockIdx.z;
+    // late query tiles visit the most chunks: launch them first, across all (b, group), so that short CTAs
+    // make the grid's tail
+    const XSlowest blk = x_slowest_block();
+    const int i0 = (gridDim.x - 1 - blk.x) * QT, g = blk.y, b = blk.z;
     const int S = D.S, K = D.topk;
     unsigned char *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     unsigned char *Qs = base, *DOs = base + kRowTile;
@@ -656,6 +658,8 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     __shared__ uint32_t s_tmem;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = D.G, QT = 128 / G;
+    // chunks in launch order within each (b, group): the concurrently running CTAs share that group's
+    // query and dO tiles in L2 (chunk-major order across the groups measured slower)
     const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int S = D.S;
     unsigned char *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);

@@ -69,7 +69,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     const int G = D.G, QT = 128 / G;
     // Late query tiles visit the most chunks (every earlier candidate): launch them first so that the
     // grid's tail is made of short CTAs.
-    const int i0 = (gridDim.x - 1 - blockIdx.x) * QT, g = blockIdx.y, b = blockIdx.z;
+    const XSlowest blk = x_slowest_block();  // across all (b, group), not within each
+    const int i0 = (gridDim.x - 1 - blk.x) * QT, g = blk.y, b = blk.z;
     const int S = D.S, K = D.topk;
     unsigned char *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     unsigned char *Qs = base;

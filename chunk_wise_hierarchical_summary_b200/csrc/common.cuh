@@ -125,6 +125,19 @@ __device__ __forceinline__ void warp_bitonic_sort(uint64_t (&v)[NPL]) {
     }
 }
 
+// Block (x, y, z) of a grid, renumbered so that x varies slowest in launch order (blocks are launched
+// with x fastest): returns the x, y and z this block works on. With work that shrinks as x grows, every
+// (y, z) slice's heaviest blocks then start first and the grid's tail is made of light ones.
+struct XSlowest {
+    int x, y, z;
+};
+__device__ __forceinline__ XSlowest x_slowest_block() {
+    const unsigned lin = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+    const unsigned nyz = gridDim.y * gridDim.z;
+    const unsigned rem = lin % nyz;
+    return XSlowest{(int)(lin / nyz), (int)(rem % gridDim.y), (int)(rem / gridDim.y)};
+}
+
 // Programmatic dependent launch: a kernel launched with launch_pdl may start while the grid before it
 // on the stream is still running; grid_dep_wait() blocks until that grid has completed and its memory
 // is visible (a no-op for an ordinary launch). Every CTA of such a kernel calls it before reading what
