@@ -3,12 +3,18 @@
 //
 // CTA = (128 query rows, KV group g, batch b); 16 warps. For each head h of the group one thread
 // TMA-loads the q^ tile [128 x 128] and the summary tile k'_h [128 chunks x 128] (128-byte swizzle,
-// two stages) and issues 8 tcgen05.mma (M 128, N 128, K 16) into TMEM columns [128h, 128h+128):
-// D[i][c] = q^_i . k'_c. Then, with rows in TMEM lanes:
-//   phase 1  warp (quadrant, head): s^ = tau D + b', masked to the row's candidates; LSE_h per row.
-//   phase 2  warp (quadrant, column block of 32): g_c = max_h (s^_{h,c} - LSE_h) as 64-bit keys
-//            (score desc, chunk id asc); each thread keeps its block's best K1 in a sorted register list.
-//   phase 3  one thread per row merges the four lists: top-k ids (ascending) and the gap.
+// three stages, the first loads issued before the setup barrier) and issues 8 tcgen05.mma (M 128, N 128,
+// K 16) into TMEM columns [128h, 128h+128): D[i][c] = q^_i . k'_c, committing one barrier per head.
+// Then, with rows in TMEM lanes:
+//   phase 1  warp (quadrant, head), as soon as its head's product has landed: s^ = tau D + b' (log2
+//            units), masked to the row's candidates; LSE_h per row, the next block's TMEM load in flight.
+//   phase 2  warp (quadrant, column block of 32): g_c = max_h (s^_{h,c} - LSE_h) as 32-bit keys (score
+//            desc cut to 16 mantissa bits, chunk id asc), sorted by a register bitonic network; the
+//            exact scores go to shared memory for the gap.
+//   phase 3  four lanes of a warp merge a row's four lists (two shuffles a step): top-k ids (ascending,
+//            from a 128-bit mask) and the gap, staged in shared memory.
+//   phase 4  (optional) each head's s^ of the selected ids, staged in shared memory.
+// Ids and scores leave in coalesced copies (the CTA's rows are contiguous).
 // Rows whose candidates exceed 128 chunks use the general kernel (select.cu).
 //
 // Fused Q-Cal (Sec. 4, q^ = q + W_up W_down h with h = q and one rank-32 pair for all heads): the
