@@ -76,7 +76,9 @@ def _load() -> ctypes.CDLL:
     lib.hils_check.restype = st
     lib.hils_status_string.argtypes = [st]
     lib.hils_status_string.restype = ctypes.c_char_p
+    lib.hils_last_error.argtypes = []
     lib.hils_last_error.restype = ctypes.c_char_p
+    lib.hils_version.argtypes = []
     lib.hils_version.restype = ctypes.c_char_p
     return lib
 

@@ -28,6 +28,48 @@ def test_every_declared_symbol_is_exported():
     assert exported == set(names)
 
 
+def _header_prototypes():
+    """(return type, [parameter types]) of every HILS_API function, comments stripped."""
+    text = open(os.path.join(ROOT, "include", "hils.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    protos = {}
+    for m in re.finditer(r"HILS_API\s+([\w\s\*]*?)\b(hils_\w+)\s*\(([^;{)]*)\)\s*;", text):
+        ret, name, args = " ".join(m.group(1).split()), m.group(2), m.group(3).strip()
+        params = [] if args in ("", "void") else [re.sub(r"\b\w+$", "", " ".join(a.split())).strip()
+                                                  for a in args.split(",")]
+        protos[name] = (ret, params)
+    return protos
+
+
+def _ctype_for(c_type: str):
+    """The ctypes type the binding must give a header type: pointers and streams as void pointers, the
+    params struct by pointer, integers by their width and sign, status enums as int."""
+    if c_type == "const hils_params *":
+        return ctypes.POINTER(H.Params)
+    if c_type.endswith("*") or c_type == "hils_stream_t":
+        return ctypes.c_void_p
+    return {"size_t": ctypes.c_size_t, "int32_t": ctypes.c_int32, "int": ctypes.c_int,
+            "uint32_t": ctypes.c_uint32, "hils_status": ctypes.c_int}[c_type]
+
+
+def test_binding_signatures_match_the_header():
+    protos = _header_prototypes()
+    assert set(protos) == set(H.EXPORTED)
+    for name, (ret, params) in protos.items():
+        f = getattr(H.lib, name)
+        assert f.argtypes is not None, name
+        assert len(f.argtypes) == len(params), name
+        for i, (have, c_type) in enumerate(zip(f.argtypes, params)):
+            assert have == _ctype_for(c_type), (name, i, c_type, have)
+        want = ctypes.c_char_p if ret == "const char *" else _ctype_for(ret)
+        assert f.restype == want, (name, ret, f.restype)
+    # the params struct: ten int32 sizes, the float scale, the int32 dtype, in the header's order
+    assert [n for n, _ in H.Params._fields_] == ["B", "T", "L", "Hq", "Hkv", "d", "S", "topk", "window",
+                                                 "q_pos0", "scale", "dtype"]
+    assert ctypes.sizeof(H.Params) == 12 * 4
+
+
 def test_status_strings_and_version():
     for code, name in H.STATUS.items():
         assert H.lib.hils_status_string(code).decode() == name
