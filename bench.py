@@ -200,9 +200,11 @@ METRIC = ("HiLS prefill tokens/s (B4 T8192 Hq16 Hkv4 d128 S64 k16 W512); decode 
 
 
 # DRAM bytes (read + write) of one attn_tc_kernel launch at the prefill workload, from one ncu capture
-# (`--metrics dram__bytes_read.sum,dram__bytes_write.sum` of `bench.py --profile attn`): 241.7 MB read,
-# 102.2 MB written. Valid for the kernel as captured; set to None when the kernel changes.
-ATTN_TC_TRAFFIC_BYTES = 241742336 + 102183680
+# (`--metrics dram__bytes_read.sum,dram__bytes_write.sum` of `bench.py --profile attn`), or None when the
+# kernel has changed since that capture. The last capture (241.7 MB read, 102.2 MB written: the inputs
+# read once) predates the kernel's launch order across (batch, KV group), so the line reports None.
+ATTN_TC_TRAFFIC_BYTES = None
+ATTN_TC_LAST_CAPTURE_BYTES = 241742336 + 102183680
 
 
 def base_config(w: W.Workload, world: int) -> dict:
@@ -300,7 +302,10 @@ def bench_prefill(args, dist, dev, H, peaks):
                      "traffic": ATTN_TC_TRAFFIC_BYTES,
                      "note": "algorithmic flops = 4*d per (row, head, attended token); attended = window + "
                              "selected chunk tokens, %.1f per query on average; traffic = DRAM bytes per "
-                             "attn_tc_kernel launch (ncu)" % work["avg_attended"]},
+                             "attn_tc_kernel launch (ncu)%s" % (
+                                 work["avg_attended"], "" if ATTN_TC_TRAFFIC_BYTES is not None else
+                                 ", null: the kernel's launch order changed after its last capture (%.1f MB per "
+                                 "launch, the inputs read once)" % (ATTN_TC_LAST_CAPTURE_BYTES / 1e6))},
         "launches_per_step": 3,
     }
     del flush
