@@ -113,6 +113,21 @@ def _stream(device) -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
+def _lead(name, t, ndim):
+    """Device and dtype of a call's leading tensor, the one its sizes are read from: a contiguous CUDA
+    tensor with ndim dimensions. The library launches on the current CUDA device, so every call runs
+    with this tensor's device current (torch.cuda.device around the C call)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} has {t.dim()} dimensions, expected {ndim}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} is on {t.device}: the library takes CUDA tensors only")
+    return t.device, t.dtype
+
+
 def _check(name, t, dtype, shape, device):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
@@ -141,9 +156,9 @@ def chunk_summary(k, q_land, S: int, *, c_begin: int = 0, c_end: int | None = No
                   scale: float = 0.0):
     """Eq. 8 summaries. k [B,Hkv,L,d], q_land [B,Hq,Nc,d] -> (k_sum [B,Hq,Nc,d], b_sum [B,Hq,Nc] fp32).
     With c_begin/c_end only those chunks are (re)computed into the given k_sum/b_sum."""
+    dev, dt = _lead("k", k, 4)
     B, Hkv, L, d = k.shape
     Hq, Nc = q_land.shape[1], q_land.shape[2]
-    dev, dt = k.device, k.dtype
     _check("q_land", q_land, dt, (B, Hq, L // S, d), dev)
     if k_sum is None:
         k_sum = torch.empty((B, Hq, Nc, d), dtype=dt, device=dev)
@@ -154,8 +169,9 @@ def chunk_summary(k, q_land, S: int, *, c_begin: int = 0, c_end: int | None = No
     _check("k", k, dt, (B, Hkv, L, d), dev)
     p = make_params(B, 1, L, Hq, Hkv, d, S, 1, 1, 0, scale, dt)
     c_end = Nc if c_end is None else c_end
-    _raise(lib.hils_chunk_summary(ctypes.byref(p), _ptr(k), _ptr(q_land), c_begin, c_end, _ptr(k_sum), _ptr(b_sum),
-                                  _stream(dev)))
+    with torch.cuda.device(dev):
+        _raise(lib.hils_chunk_summary(ctypes.byref(p), _ptr(k), _ptr(q_land), c_begin, c_end, _ptr(k_sum), _ptr(b_sum),
+                                      _stream(dev)))
     return k_sum, b_sum
 
 
@@ -163,9 +179,9 @@ def chunk_summary_shared_query(k, q_shared, S: int, *, c_begin: int = 0, c_end: 
                                b_sum=None, scale: float = 0.0):
     """Eq. 8 summaries with one shared landmark query per head (Sec. 4): k [B,Hkv,L,d], q_shared [Hq,d]
     -> (k_sum [B,Hq,Nc,d], b_sum [B,Hq,Nc] fp32), as chunk_summary with q_land[b,h,c] = q_shared[h]."""
+    dev, dt = _lead("k", k, 4)
     B, Hkv, L, d = k.shape
     Hq, Nc = q_shared.shape[0], L // S
-    dev, dt = k.device, k.dtype
     _check("q_shared", q_shared, dt, (Hq, d), dev)
     if k_sum is None:
         k_sum = torch.empty((B, Hq, Nc, d), dtype=dt, device=dev)
@@ -176,8 +192,9 @@ def chunk_summary_shared_query(k, q_shared, S: int, *, c_begin: int = 0, c_end: 
     _check("k", k, dt, (B, Hkv, L, d), dev)
     p = make_params(B, 1, L, Hq, Hkv, d, S, 1, 1, 0, scale, dt)
     c_end = Nc if c_end is None else c_end
-    _raise(lib.hils_chunk_summary_shared_query(ctypes.byref(p), _ptr(k), _ptr(q_shared), c_begin, c_end, _ptr(k_sum),
-                                               _ptr(b_sum), _stream(dev)))
+    with torch.cuda.device(dev):
+        _raise(lib.hils_chunk_summary_shared_query(ctypes.byref(p), _ptr(k), _ptr(q_shared), c_begin, c_end,
+                                                   _ptr(k_sum), _ptr(b_sum), _stream(dev)))
     return k_sum, b_sum
 
 
@@ -208,16 +225,17 @@ def select_topk(q_hat, k_sum, b_sum, *, Hkv: int, L: int, S: int, topk: int, win
     """GQA-shared top-k (Eq. 7, Sec. 3 RQ1, Sec. 4). q_hat [B,Hq,T,d], k_sum [B,Hq,Nc,d], b_sum [B,Hq,Nc]
     -> idx [B,Hkv,T,topk] int32 (ascending ids, -1 padded); with with_gap also gap [B,Hkv,T] fp32 and with
     with_shat (idx, gap or None, shat [B,Hq,T,topk] fp32: each head's s^ of the selected ids)."""
+    dev, dt = _lead("q_hat", q_hat, 4)
     B, Hq, T, d = q_hat.shape
-    dev, dt = q_hat.device, q_hat.dtype
     Nc = L // S
     _check("k_sum", k_sum, dt, (B, Hq, Nc, d), dev)
     _check("b_sum", b_sum, torch.float32, (B, Hq, Nc), dev)
     idx, gap, shat = _selection_outputs(B, Hq, Hkv, T, topk, dev, with_gap, with_shat, idx, gap, shat)
     p = make_params(B, T, L, Hq, Hkv, d, S, topk, window, q_pos0, scale, dt)
     ws, nws = _workspace(p, OP_SELECT, dev, None)
-    _raise(lib.hils_select_topk(ctypes.byref(p), _ptr(q_hat), _ptr(k_sum), _ptr(b_sum), _ptr(idx), _ptr(gap),
-                                _ptr(shat), _ptr(ws), nws, _stream(dev)))
+    with torch.cuda.device(dev):
+        _raise(lib.hils_select_topk(ctypes.byref(p), _ptr(q_hat), _ptr(k_sum), _ptr(b_sum), _ptr(idx), _ptr(gap),
+                                    _ptr(shat), _ptr(ws), nws, _stream(dev)))
     return _selection_result(idx, gap, shat, with_shat)
 
 
@@ -226,8 +244,8 @@ def select_topk_qcal(q, w_down, w_up, k_sum, b_sum, *, Hkv: int, L: int, S: int,
                      gap=None, shat=None):
     """select_topk with Q-Cal fused (Sec. 4): q [B,Hq,T,d], w_down [r,d], w_up [d,r] (r = 32) ->
     idx [B,Hkv,T,topk] int32 (and gap, shat as select_topk), selected on q^ = q + W_up (W_down q)."""
+    dev, dt = _lead("q", q, 4)
     B, Hq, T, d = q.shape
-    dev, dt = q.device, q.dtype
     r = w_down.shape[0]
     _check("w_down", w_down, dt, (r, d), dev)
     _check("w_up", w_up, dt, (d, r), dev)
@@ -236,8 +254,9 @@ def select_topk_qcal(q, w_down, w_up, k_sum, b_sum, *, Hkv: int, L: int, S: int,
     _check("b_sum", b_sum, torch.float32, (B, Hq, Nc), dev)
     idx, gap, shat = _selection_outputs(B, Hq, Hkv, T, topk, dev, with_gap, with_shat, idx, gap, shat)
     p = make_params(B, T, L, Hq, Hkv, d, S, topk, window, q_pos0, scale, dt)
-    _raise(lib.hils_select_topk_qcal(ctypes.byref(p), _ptr(q), _ptr(w_down), _ptr(w_up), r, _ptr(k_sum), _ptr(b_sum),
-                                     _ptr(idx), _ptr(gap), _ptr(shat), _stream(dev)))
+    with torch.cuda.device(dev):
+        _raise(lib.hils_select_topk_qcal(ctypes.byref(p), _ptr(q), _ptr(w_down), _ptr(w_up), r, _ptr(k_sum),
+                                         _ptr(b_sum), _ptr(idx), _ptr(gap), _ptr(shat), _stream(dev)))
     return _selection_result(idx, gap, shat, with_shat)
 
 
@@ -246,9 +265,9 @@ def bsa_select_topk(q, k, *, S: int, topk: int, window: int, q_pos0: int = 0, sc
     """Naive BSA selection (Sec. 2): exact chunk log-masses and the GQA top-k on them. q [B,Hq,T,d],
     k [B,Hkv,L,d] -> (idx [B,Hkv,T,topk] int32, gap [B,Hkv,T] fp32 or None, mass [B,Hq,T,Nc] fp32; entries
     of mass at c >= n_i are not written)."""
+    dev, dt = _lead("q", q, 4)
     B, Hq, T, d = q.shape
     Hkv, L = k.shape[1], k.shape[2]
-    dev, dt = q.device, q.dtype
     Nc = L // S
     _check("k", k, dt, (B, Hkv, L, d), dev)
     if idx is None:
@@ -262,18 +281,19 @@ def bsa_select_topk(q, k, *, S: int, topk: int, window: int, q_pos0: int = 0, sc
         mass = torch.empty((B, Hq, T, Nc), dtype=torch.float32, device=dev)
     _check("mass", mass, torch.float32, (B, Hq, T, Nc), dev)
     p = make_params(B, T, L, Hq, Hkv, d, S, topk, window, q_pos0, scale, dt)
-    _raise(lib.hils_bsa_select_topk(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(idx), _ptr(gap), _ptr(mass),
-                                    _stream(dev)))
+    with torch.cuda.device(dev):
+        _raise(lib.hils_bsa_select_topk(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(idx), _ptr(gap), _ptr(mass),
+                                        _stream(dev)))
     return idx, gap, mass
 
 
 def attn_fwd(q, k, v, q_hat, k_sum, b_sum, idx, *, S: int, window: int, q_pos0: int = 0, scale: float = 0.0,
              out=None, lse=None, workspace=None):
     """Eq. 10 prefill. q, q_hat [B,Hq,T,d]; k, v [B,Hkv,L,d]; idx [B,Hkv,T,topk] -> out [B,Hq,T,d], lse [B,Hq,T]."""
+    dev, dt = _lead("q", q, 4)
     B, Hq, T, d = q.shape
     Hkv, L = k.shape[1], k.shape[2]
     topk = idx.shape[-1]
-    dev, dt = q.device, q.dtype
     Nc = L // S
     for name, t, shape in (("k", k, (B, Hkv, L, d)), ("v", v, (B, Hkv, L, d)), ("q_hat", q_hat, (B, Hq, T, d)),
                            ("k_sum", k_sum, (B, Hq, Nc, d))):
@@ -288,8 +308,9 @@ def attn_fwd(q, k, v, q_hat, k_sum, b_sum, idx, *, S: int, window: int, q_pos0: 
     _check("lse", lse, torch.float32, (B, Hq, T), dev)
     p = make_params(B, T, L, Hq, Hkv, d, S, topk, window, q_pos0, scale, dt)
     ws, nws = _workspace(p, OP_ATTN_FWD, dev, workspace)
-    _raise(lib.hils_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_hat), _ptr(k_sum), _ptr(b_sum),
-                             _ptr(idx), _ptr(out), _ptr(lse), _ptr(ws), nws, _stream(dev)))
+    with torch.cuda.device(dev):
+        _raise(lib.hils_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_hat), _ptr(k_sum), _ptr(b_sum),
+                                 _ptr(idx), _ptr(out), _ptr(lse), _ptr(ws), nws, _stream(dev)))
     return out, lse
 
 
@@ -297,10 +318,10 @@ def attn_fwd_shat(q, k, v, idx, shat, *, S: int, window: int, q_pos0: int = 0, s
                   lse=None):
     """Eq. 10 prefill from the selection's ids and retrieval scores (select_topk with_shat). q [B,Hq,T,d];
     k, v [B,Hkv,L,d]; idx [B,Hkv,T,topk] canonical; shat [B,Hq,T,topk] -> out [B,Hq,T,d], lse [B,Hq,T]."""
+    dev, dt = _lead("q", q, 4)
     B, Hq, T, d = q.shape
     Hkv, L = k.shape[1], k.shape[2]
     topk = idx.shape[-1]
-    dev, dt = q.device, q.dtype
     for name, t, shape in (("k", k, (B, Hkv, L, d)), ("v", v, (B, Hkv, L, d))):
         _check(name, t, dt, shape, dev)
     _check("idx", idx, torch.int32, (B, Hkv, T, topk), dev)
@@ -312,8 +333,9 @@ def attn_fwd_shat(q, k, v, idx, shat, *, S: int, window: int, q_pos0: int = 0, s
     _check("out", out, dt, (B, Hq, T, d), dev)
     _check("lse", lse, torch.float32, (B, Hq, T), dev)
     p = make_params(B, T, L, Hq, Hkv, d, S, topk, window, q_pos0, scale, dt)
-    _raise(lib.hils_attn_fwd_shat(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(shat), _ptr(out),
-                                  _ptr(lse), _stream(dev)))
+    with torch.cuda.device(dev):
+        _raise(lib.hils_attn_fwd_shat(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(shat), _ptr(out),
+                                      _ptr(lse), _stream(dev)))
     return out, lse
 
 
@@ -323,9 +345,9 @@ def decode(q, q_hat, k_cache, v_cache, k_sum, b_sum, *, S: int, topk: int, windo
     q, q_hat [B,Hq,M,d]; caches [B,Hkv,L,d]; k_sum [B,Hq,Nc,d]; b_sum [B,Hq,Nc] -> out [B,Hq,M,d],
     lse [B,Hq] for M = 1 else [B,Hq,M] (and idx [B,Hkv,topk] for M = 1 else [B,Hkv,M,topk] with
     return_idx)."""
+    dev, dt = _lead("q", q, 4)
     B, Hq, M, d = q.shape
     Hkv, L = k_cache.shape[1], k_cache.shape[2]
-    dev, dt = q.device, q.dtype
     Nc = L // S
     _check("q", q, dt, (B, Hq, M, d), dev)
     _check("q_hat", q_hat, dt, (B, Hq, M, d), dev)
@@ -347,18 +369,19 @@ def decode(q, q_hat, k_cache, v_cache, k_sum, b_sum, *, S: int, topk: int, windo
         _check("idx_out", idx_out, torch.int32, idx_shape, dev)
     p = make_params(B, M, L, Hq, Hkv, d, S, topk, window, L - M, scale, dt)
     ws, nws = _workspace(p, OP_DECODE, dev, workspace)
-    _raise(lib.hils_decode(ctypes.byref(p), _ptr(q), _ptr(q_hat), _ptr(k_cache), _ptr(v_cache), _ptr(k_sum),
-                           _ptr(b_sum), _ptr(out), _ptr(lse), _ptr(idx_out), _ptr(ws), nws, _stream(dev)))
+    with torch.cuda.device(dev):
+        _raise(lib.hils_decode(ctypes.byref(p), _ptr(q), _ptr(q_hat), _ptr(k_cache), _ptr(v_cache), _ptr(k_sum),
+                               _ptr(b_sum), _ptr(out), _ptr(lse), _ptr(idx_out), _ptr(ws), nws, _stream(dev)))
     return (out, lse, idx_out) if idx_out is not None else (out, lse)
 
 
 def attn_bwd(q, k, v, q_hat, q_land, k_sum, b_sum, idx, out, lse, dout, *, S: int, window: int, scale: float = 0.0,
              workspace=None):
     """Gradients of sum(dout * out) with idx fixed -> (dq, dk, dv, dq_hat, dq_land)."""
+    dev, dt = _lead("q", q, 4)
     B, Hq, T, d = q.shape
     Hkv, L = k.shape[1], k.shape[2]
     topk = idx.shape[-1]
-    dev, dt = q.device, q.dtype
     Nc = L // S
     for name, t, shape in (("k", k, (B, Hkv, L, d)), ("v", v, (B, Hkv, L, d)), ("q_hat", q_hat, (B, Hq, T, d)),
                            ("q_land", q_land, (B, Hq, Nc, d)), ("k_sum", k_sum, (B, Hq, Nc, d)),
@@ -372,16 +395,18 @@ def attn_bwd(q, k, v, q_hat, q_land, k_sum, b_sum, idx, out, lse, dout, *, S: in
     dq_land = torch.empty_like(q_land)
     p = make_params(B, T, L, Hq, Hkv, d, S, topk, window, 0, scale, dt)
     ws, nws = _workspace(p, OP_ATTN_BWD, dev, workspace)
-    _raise(lib.hils_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_hat), _ptr(q_land), _ptr(k_sum),
-                             _ptr(b_sum), _ptr(idx), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
-                             _ptr(dq_hat), _ptr(dq_land), _ptr(ws), nws, _stream(dev)))
+    with torch.cuda.device(dev):
+        _raise(lib.hils_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_hat), _ptr(q_land), _ptr(k_sum),
+                                 _ptr(b_sum), _ptr(idx), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                 _ptr(dq_hat), _ptr(dq_land), _ptr(ws), nws, _stream(dev)))
     return dq, dk, dv, dq_hat, dq_land
 
 
 def check(device=None) -> None:
     """Synchronise the current stream and raise on a CUDA or device-side error."""
-    dev = device or torch.device("cuda", torch.cuda.current_device())
-    _raise(lib.hils_check(_stream(dev)))
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):  # the error words read are those of the current device
+        _raise(lib.hils_check(_stream(dev)))
 
 
 def prefill(q, k, v, q_hat, q_land, *, S: int, topk: int, window: int, scale: float = 0.0):
