@@ -1,5 +1,6 @@
 """Host logic of bench.py that needs no GPU: the algorithmic byte and flop counts behind the roofline
-fractions, and the line both arms print."""
+fractions, the attention's packing statistic, the clock summary that decides whether a run is kept, and
+the line both arms print."""
 import os
 import sys
 
@@ -83,3 +84,40 @@ def test_reference_arm_line_matches_the_gpu_arms_config_and_sample(capsys):
     assert line["config"] == bench.base_config(W.PREFILL_BF16, 1)
     assert line["cpu_baseline"]["sample"].startswith(bench.oracle_sample_text(W.PREFILL_BF16, 1))
     assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
+
+
+def test_packing_counts_selected_chunks_per_query_and_distinct_chunks_per_tile():
+    # G = 4: a tile packs 32 queries. Tile 0: every query selects chunks {0, 1}. Tile 1: even queries
+    # select {2, 3}, odd queries {4} (one id, then -1 padding).
+    w = W.Workload("pack", B=1, T=64, L=512, Hq=4, Hkv=1, d=64, S=64, topk=2, W=64, dtype="fp32", recipe="scaled")
+    idx = torch.empty((1, 1, 64, 2), dtype=torch.int32)
+    idx[0, 0, :32] = torch.tensor([0, 1], dtype=torch.int32)
+    idx[0, 0, 32::2] = torch.tensor([2, 3], dtype=torch.int32)
+    idx[0, 0, 33::2] = torch.tensor([4, -1], dtype=torch.int32)
+    s = bench.packing_stats(w, idx)
+    assert s["queries_per_tile"] == 32
+    assert s["selected_chunks_per_query"] == (32 * 2 + 16 * 2 + 16 * 1) / 64
+    assert s["selected_chunks_per_tile"] == (2 + 3) / 2
+
+
+def test_clock_summary_reads_median_max_and_active_reasons():
+    idle = "0, 1965, 1965, 650.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active\n"
+    capped = "0, 1950, 1965, 990.5, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n"
+    hot = "0, 1200, 1965, 500.0, 0x0000000000000048, Not Active, Active, Not Active, Not Active\n"
+    assert bench.summarise_clocks([idle, capped, idle, "a partial line, 1965\n"]) == {
+        "sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    s = bench.summarise_clocks([idle, hot])
+    assert s["reasons"] == ["hw_thermal_slowdown"] and s["sm_mhz"] == (1965.0 + 1200.0) / 2
+    assert bench.summarise_clocks([]) is None
+    na = "0, [N/A], [N/A], [N/A], [N/A], [N/A], [N/A], [N/A], [N/A]\n"
+    assert bench.summarise_clocks([na]) == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 1}
+
+
+def test_clock_sampler_watches_the_physical_gpu(monkeypatch):
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "3,5")
+    assert bench.physical_gpu_index(0) == 3 and bench.physical_gpu_index(1) == 5
+    assert bench.physical_gpu_index(2) == 2  # past the list: the local rank
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "GPU-0a1b2c3d")  # a UUID: the local rank
+    assert bench.physical_gpu_index(0) == 0
+    monkeypatch.delenv("CUDA_VISIBLE_DEVICES")
+    assert bench.physical_gpu_index(3) == 3
