@@ -70,8 +70,10 @@ class ClockSampler:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
                  "-i", str(self.gpu_index), "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
-        except OSError:
+        except OSError:  # no nvidia-smi: the line carries no clock record
             self.proc = None
+            if self.path is not None and os.path.exists(self.path):
+                os.unlink(self.path)
         return self
 
     def stop(self):

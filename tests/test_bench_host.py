@@ -121,3 +121,36 @@ def test_clock_sampler_watches_the_physical_gpu(monkeypatch):
     assert bench.physical_gpu_index(0) == 0
     monkeypatch.delenv("CUDA_VISIBLE_DEVICES")
     assert bench.physical_gpu_index(3) == 3
+
+
+def test_clock_sampler_reads_and_removes_its_csv(monkeypatch):
+    class FakeSmi:  # writes two rows to the file nvidia-smi is asked for, then waits to be stopped
+        def __init__(self, cmd, stdout=None, stderr=None):
+            self.path = cmd[cmd.index("-f") + 1]
+            assert cmd[cmd.index("-i") + 1] == "2" and cmd[0] == "nvidia-smi"
+            with open(self.path, "w") as f:
+                f.write("2, 1965, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, Not Active\n"
+                        "2, 1935, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active\n")
+            self.stopped = False
+
+        def terminate(self):
+            self.stopped = True
+
+        def wait(self, timeout=None):
+            assert self.stopped
+            return 0
+
+    monkeypatch.setattr(bench.subprocess, "Popen", FakeSmi)
+    monkeypatch.setattr(bench.time, "sleep", lambda s: None)
+    sampler = bench.ClockSampler(2).start()
+    path = sampler.path
+    assert sampler.stop() == {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 2}
+    assert not os.path.exists(path)
+
+    def no_smi(*a, **k):
+        raise FileNotFoundError("nvidia-smi")
+
+    monkeypatch.setattr(bench.subprocess, "Popen", no_smi)
+    sampler = bench.ClockSampler(0).start()
+    assert not os.path.exists(sampler.path)  # its temporary file is not left behind
+    assert sampler.stop() is None  # no sampler: the line carries no clock record
