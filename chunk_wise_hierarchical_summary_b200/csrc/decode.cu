@@ -1,7 +1,9 @@
-// Single-token decode over a long KV cache: stages (b)-(d) for one query at position L-1
-// ("Hierarchical Sparse Attention Done Right", Eq. 7, Sec. 3 RQ1, Sec. 4 "GQA", Eq. 10).
+// Decode over a long KV cache: stages (b)-(d) for the last M <= 8 query positions, each query with its own
+// window and selection (M = 1: the token at L-1) ("Hierarchical Sparse Attention Done Right", Eq. 7,
+// Sec. 3 RQ1, Sec. 4 "GQA", Eq. 10).
 //
-// Three launches (the score grid also clears the two counter arrays the later grids count with):
+// Three launches (the score grid also clears the two counter arrays the later grids count with; for
+// M > 1 the score grid is decode_score_mma.cu's, which reads every summary row once for the M queries):
 //  1. score    persistent, one CTA per SM: a producer lane keeps a ring of bulk copies of 128-candidate
 //              summary slices (32 KiB at d 128 bf16) in flight; consumer warps compute
 //              s^_{h,c} = tau q^_h . k'_{h,c} + b'_{h,c} into a score buffer plus per-warp partials
@@ -10,9 +12,9 @@
 //              g_c = max_h (s^_{h,c} - LSE_h) as 64-bit keys (score desc, chunk id asc), top-k. For
 //              topk <= 32 and G <= 8 one CTA per group: up to 2048 candidates, each of eight warps sorts
 //              its 256 keys in registers and warp 0 merges their best 32; longer lists keep an exact
-//              lower bound of the top-k and sort the few candidates at or below it. With few groups and
-//              very long lists several CTAs per group keep their part's top-k and the last CTA to
-//              finish (atomic counter, no waiting) merges them.
+//              lower bound of the top-k and rank the few candidates at or below it (one thread each).
+//              With few groups and very long lists several CTAs per group keep their part's top-k and
+//              the last CTA to finish (atomic counter, no waiting) merges them.
 //  3. attend   bf16 d 128 S 64 G <= 8: decode_attn_mma.cu (split-K CTAs over the group's tiles,
 //              warp-level MMAs, online Eq. 10 merge). Otherwise here: one S-token tile (a selected
 //              chunk or a window tile) per CTA, K and V staged by bulk copies, all G heads, a partial
